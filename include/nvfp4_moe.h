@@ -1,0 +1,191 @@
+/*
+ * nvfp4_moe.h -- C ABI of the B200 (sm_100a) routed mixture-of-experts FFN layer
+ * over ModelOpt-style NVFP4 expert weights.
+ *
+ * What the layer computes (per token t, top-k experts e_j, j = 0..K-1):
+ *
+ *   g   = s_g(e) * (G_e x_t)          gate projection,  G_e [I][H]
+ *   u   = s_u(e) * (U_e x_t)          up projection,    U_e [I][H]
+ *   h   = SiLU(g) * u,  SiLU(z) = z / (1 + exp(-z))
+ *   y   = s_d(e) * (D_e h)            down projection,  D_e [H][I]
+ *   out_t = sum_j w_{t,j} * y_{t,e_j}
+ *
+ * Sources on the pages:
+ *   - NVFP4 expert weights: 4-bit codes with a scale per group of 16 inputs and
+ *     one FP32 tensor scale ("TensorFold PR #906", first post: input cuts keep
+ *     groups of 16, the FP32 tensor scale is unchanged; "Strata NVFP4" README,
+ *     "How it differs from upstream Strata": 4.5-bit experts with calibrated
+ *     scales, lossless repack).
+ *   - The per-expert FP32 scale is applied to each projection's OUTPUT, not folded
+ *     into the operands ("Strata NVFP4" README, "How it differs", first bullet);
+ *     folding a tiny scale into FP16 activations pushed them into FP16 subnormals
+ *     (same README, the "Fixes" bullet). This library applies s_g, s_u, s_d in
+ *     FP32 after accumulation.
+ *   - Routed experts, gate/up/down tensors stacked per layer: "#2727 tools: add
+ *     opt-in FP4-Local CSF checkpoint conversion", "Validation" (144 NVFP4 expert
+ *     tensors, 512 experts each; nine projection global scales for three experts).
+ *   - One launch per expert group after one wait instead of a wait per expert:
+ *     "Strata NVFP4" README, "How it differs", the prompt-reading bullet. Every
+ *     forward call here is a fixed sequence of launches with no host read-back.
+ *   - The pages never write the routing math out. Routing here is softmax top-k,
+ *     renormalised over the K selected experts (the tiny-layer workload's
+ *     definition); this equals exp(l_j - l_max) / sum over the K selected.
+ *
+ * Packed formats (all planes row-major, no padding, no swizzle):
+ *   E2M1 code nibble: bit 3 sign, bits 2..1 exponent, bit 0 mantissa (OCP MX);
+ *     magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6. Element 2c of a row is in the LOW
+ *     nibble of byte c, element 2c+1 in the HIGH nibble.
+ *   E4M3 scale byte (OCP FP8 E4M3FN): bias 7, no infinities, 0x7F/0xFF NaN.
+ *     Scales must be finite and non-negative; the layer does not re-check them.
+ *   Weight value = code * scale[row][col/16] * global.
+ *
+ * Memory and ownership:
+ *   - Every pointer in nvfp4_moe_weights and nvfp4_moe_io is a DEVICE pointer
+ *     owned by the caller. The handle BORROWS the weight pointers: they must stay
+ *     valid until nvfp4_moe_destroy. The library allocates no device memory
+ *     except one 64-byte status block made by nvfp4_moe_create.
+ *   - All scratch lives in the caller's workspace (nvfp4_moe_workspace_bytes).
+ *
+ * Errors: every call returns 0 (NVFP4_MOE_OK) or a negative nvfp4_moe_status.
+ *   Host-side checks run before anything is enqueued; a call that fails them
+ *   enqueues nothing. Conditions found on the device (routing id out of range
+ *   or duplicated, a non-finite routing logit) are latched in the status block
+ *   and returned by nvfp4_moe_get_status. forward never synchronises.
+ *
+ * Threading: a handle may be used from one host thread at a time. Two forward
+ *   calls that run concurrently on the GPU must not share a workspace.
+ */
+#ifndef NVFP4_MOE_H
+#define NVFP4_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define NVFP4_MOE_ABI_VERSION 1
+
+/* Largest top-k the kernels support, and the largest T the decode path takes. */
+#define NVFP4_MOE_MAX_TOPK 16
+#define NVFP4_MOE_DECODE_MAX_T 8
+
+typedef enum {
+    NVFP4_MOE_OK = 0,
+    NVFP4_MOE_ERR_INVALID_ARG = -1,        /* null pointer, T<0, T>max_tokens, bad enum   */
+    NVFP4_MOE_ERR_UNSUPPORTED_DIMS = -2,   /* H or I not a multiple of 128; K>E; K>16; E>1024 */
+    NVFP4_MOE_ERR_MISALIGNED = -3,         /* a plane or buffer not 16-byte aligned       */
+    NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL = -4,
+    NVFP4_MOE_ERR_CUDA = -5,               /* a CUDA runtime/driver call failed           */
+    NVFP4_MOE_ERR_BAD_ROUTING = -6,        /* device: precomputed id out of [0,E) or repeated */
+    NVFP4_MOE_ERR_NONFINITE = -7,          /* device: a selected routing logit is NaN/inf */
+    NVFP4_MOE_ERR_TIMEOUT = -8,            /* device: a bounded wait gave up              */
+    NVFP4_MOE_ERR_NO_DEVICE = -9           /* no sm_100 device current                    */
+} nvfp4_moe_status;
+
+typedef struct nvfp4_moe nvfp4_moe_t; /* opaque handle */
+
+/* Layer geometry. hidden = H, inter = I, n_experts = E, top_k = K.
+ * max_tokens bounds T for every forward call and sizes the workspace. */
+typedef struct {
+    int32_t hidden;
+    int32_t inter;
+    int32_t n_experts;
+    int32_t top_k;
+    int32_t max_tokens;
+} nvfp4_moe_dims;
+
+/* Packed expert planes, DEVICE pointers, BORROWED (see above). Each code and
+ * scale plane must be 16-byte aligned; the globals 4-byte aligned.
+ *   gate_codes, up_codes   [E][I][H/2]  u8, two E2M1 codes per byte
+ *   gate_scales, up_scales [E][I][H/16] E4M3 bytes, one per 16 inputs
+ *   gate_global, up_global [E]          f32
+ *   down_codes             [E][H][I/2]
+ *   down_scales            [E][H][I/16]
+ *   down_global            [E]                                            */
+typedef struct {
+    const uint8_t *gate_codes;
+    const uint8_t *up_codes;
+    const uint8_t *gate_scales;
+    const uint8_t *up_scales;
+    const float *gate_global;
+    const float *up_global;
+    const uint8_t *down_codes;
+    const uint8_t *down_scales;
+    const float *down_global;
+} nvfp4_moe_weights;
+
+typedef enum {
+    NVFP4_MOE_ACT_BF16 = 0, /* act is [T][H] bf16                                */
+    NVFP4_MOE_ACT_INT8 = 1  /* act is [T][H] int8 q, x = q * act_scale[t] (f32) */
+} nvfp4_moe_act;
+
+typedef enum {
+    NVFP4_MOE_OUT_F32 = 0,     /* out[T][H] f32 = MoE(x)                          */
+    NVFP4_MOE_OUT_F32_ADD = 1  /* out[T][H] f32 += MoE(x)  (residual stream)       */
+} nvfp4_moe_out;
+
+/* One forward call. DEVICE pointers, caller-owned.
+ *   T               number of tokens, 0 <= T <= dims.max_tokens (T = 0 is a no-op)
+ *   act, act_scale  activations; act_scale only for NVFP4_MOE_ACT_INT8
+ *   router_logits   [T][E] f32; when NULL, topk_ids [T][K] i32 and
+ *                   topk_weights [T][K] f32 are used as given
+ *   out             [T][H] f32, written (OUT_F32) or accumulated into (OUT_F32_ADD)
+ *   dbg_*           optional (may be NULL) copies of the routing results:
+ *                   dbg_ids [T][K] i32, dbg_w [T][K] f32 (renormalised weights),
+ *                   dbg_counts [E] i32 (pairs per expert), dbg_offsets [E+1] i32
+ *                   (exclusive scan of counts), dbg_perm [T*K] i32 (pair index
+ *                   t*K+j, grouped by expert ascending, then token ascending).  */
+typedef struct {
+    int32_t T;
+    nvfp4_moe_act act_type;
+    const void *act;
+    const float *act_scale;
+    const float *router_logits;
+    const int32_t *topk_ids;
+    const float *topk_weights;
+    nvfp4_moe_out out_type;
+    float *out;
+    int32_t *dbg_ids;
+    float *dbg_w;
+    int32_t *dbg_counts;
+    int32_t *dbg_offsets;
+    int32_t *dbg_perm;
+} nvfp4_moe_io;
+
+/* Validates dims and weight pointers (all checks before any allocation), then
+ * allocates the handle and its 64-byte device status block on the current device.
+ * On failure *out is set to NULL and nothing stays allocated. Requires an sm_100
+ * device to be current. */
+int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
+                     const nvfp4_moe_weights *weights);
+
+/* Bytes of workspace a forward call with T tokens needs (256-byte aligned start
+ * required). Returns 0 for a NULL handle or T outside [0, max_tokens]. */
+size_t nvfp4_moe_workspace_bytes(const nvfp4_moe_t *h, int32_t T);
+
+/* Enqueues the whole layer on `stream` (a cudaStream_t; NULL = legacy default
+ * stream). Asynchronous: never synchronises and never reads device memory back.
+ * The workspace must not be used by another call until this one has finished
+ * on the GPU. */
+int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *workspace,
+                      size_t workspace_bytes, void *stream);
+
+/* Synchronises `stream`, returns the first device-side error latched since the
+ * last call (0 if none) and clears it. */
+int nvfp4_moe_get_status(nvfp4_moe_t *h, void *stream);
+
+/* Frees the handle and its status block. Never touches the borrowed weights. */
+void nvfp4_moe_destroy(nvfp4_moe_t *h);
+
+/* Static string for a status code. */
+const char *nvfp4_moe_strerror(int status);
+
+/* ABI version compiled into the library (NVFP4_MOE_ABI_VERSION). */
+int nvfp4_moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_MOE_H */

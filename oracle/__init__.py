@@ -1,0 +1,223 @@
+"""FP64 CPU oracle for the routed NVFP4 MoE layer -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the bench's CPU-baseline leg may
+import this package. The layer's CUDA path never does, and shares no code with it.
+
+``liboracle.so`` is built from ``nvfp4_moe_oracle.c`` with the host C compiler
+(``build()``); this module wraps it with ctypes and numpy.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nvfp4_moe_oracle.c")
+_HDR = os.path.join(_HERE, "nvfp4_moe_oracle.h")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+PLANT = {"none": 0, "nibble_order": 1, "group_shift": 2, "no_global": 3,
+         "swap_gate_up": 4, "silu_sign": 5, "equal_weights": 6}
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so (plain C, -O2, no fast-math: IEEE FP64 throughout)."""
+    stale = (not os.path.exists(_LIB) or
+             os.path.getmtime(_LIB) < max(os.path.getmtime(_SRC), os.path.getmtime(_HDR)))
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fPIC",
+                               "-shared", "-std=c11", "-D_GNU_SOURCE", "-o", tmp, _SRC,
+                               "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Dims(C.Structure):
+    _fields_ = [("E", C.c_int32), ("H", C.c_int32), ("I", C.c_int32), ("K", C.c_int32)]
+
+
+class _Weights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in (
+        "gate_codes", "up_codes", "gate_scales", "up_scales", "gate_global", "up_global",
+        "down_codes", "down_scales", "down_global")]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = C.CDLL(build())
+        _lib.orc_e2m1.restype = C.c_double
+        _lib.orc_e4m3.restype = C.c_double
+        _lib.orc_bf16.restype = C.c_double
+        _lib.orc_bf16.argtypes = [C.c_uint16]
+        _lib.orc_bf16_rne.restype = C.c_uint16
+        _lib.orc_bf16_rne.argtypes = [C.c_double]
+        _lib.orc_route.restype = C.c_int
+        _lib.orc_check_ids.restype = C.c_int
+        _lib.orc_quantize.restype = C.c_int
+        _lib.orc_moe.restype = C.c_int
+        _lib.orc_pair_h.restype = C.c_int
+        _lib.orc_pair_h.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_float,
+                                    C.c_int32, C.c_void_p, C.c_int32]
+        _lib.orc_decode_matrix.argtypes = [C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
+                                           C.c_float, C.c_void_p]
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return C.c_void_p(a.ctypes.data)
+
+
+def _np(t):
+    """torch tensor or numpy array -> contiguous numpy array on the host."""
+    if hasattr(t, "detach"):
+        t = t.detach().cpu()
+        if str(t.dtype) == "torch.bfloat16":
+            import torch
+            t = t.view(torch.int16)
+        t = t.contiguous().numpy()
+    return np.ascontiguousarray(t)
+
+
+def e2m1(nib: int) -> float:
+    return lib().orc_e2m1(C.c_uint32(nib))
+
+
+def e4m3(byte: int) -> float:
+    return lib().orc_e4m3(C.c_uint32(byte))
+
+
+def bf16(bits: int) -> float:
+    return lib().orc_bf16(C.c_uint16(bits))
+
+
+def bf16_rne(v: float) -> int:
+    return lib().orc_bf16_rne(C.c_double(v))
+
+
+def route(logits, K: int):
+    """-> (ids int32 [T][K], w float64 [T][K], n_nonfinite_tokens)"""
+    l = _np(logits).astype(np.float32, copy=False)
+    T, E = l.shape
+    ids = np.zeros((T, K), np.int32)
+    w = np.zeros((T, K), np.float64)
+    bad = lib().orc_route(C.c_int32(T), C.c_int32(E), C.c_int32(K), _p(l), _p(ids), _p(w))
+    return ids, w, bad
+
+
+def check_ids(ids, E: int) -> int:
+    i = _np(ids).astype(np.int32, copy=False)
+    T, K = i.shape
+    return lib().orc_check_ids(C.c_int32(T), C.c_int32(E), C.c_int32(K), _p(i))
+
+
+def sort(ids, E: int):
+    """-> (counts [E], offsets [E+1], perm [T*K]) int32"""
+    i = _np(ids).astype(np.int32, copy=False)
+    T, K = i.shape
+    counts = np.zeros(E, np.int32)
+    offsets = np.zeros(E + 1, np.int32)
+    perm = np.zeros(T * K, np.int32)
+    lib().orc_sort(C.c_int32(T), C.c_int32(E), C.c_int32(K), _p(i), _p(counts), _p(offsets),
+                   _p(perm))
+    return counts, offsets, perm
+
+
+def quantize(w_bf16):
+    """BF16 weights [n][rows][cols] (torch bf16 or uint16/int16 bits) ->
+    (codes u8 [n][rows][cols/2], scales u8 [n][rows][cols/16], glob f32 [n])."""
+    w = _np(w_bf16).view(np.uint16)
+    if w.ndim == 2:
+        w = w[None]
+    n, rows, cols = w.shape
+    codes = np.zeros((n, rows, cols // 2), np.uint8)
+    scales = np.zeros((n, rows, cols // 16), np.uint8)
+    glob = np.zeros(n, np.float32)
+    rc = lib().orc_quantize(C.c_int32(n), C.c_int32(rows), C.c_int32(cols), _p(w), _p(codes),
+                            _p(scales), _p(glob))
+    assert rc == 0
+    return codes, scales, glob
+
+
+def decode_matrix(codes, scales, glob) -> np.ndarray:
+    c, s = _np(codes), _np(scales)
+    rows, cols = c.shape[0], c.shape[1] * 2
+    out = np.zeros((rows, cols), np.float64)
+    lib().orc_decode_matrix(C.c_int32(rows), C.c_int32(cols), _p(c), _p(s), C.c_float(float(glob)),
+                            _p(out))
+    return out
+
+
+class _Bound:
+    """ctypes views of one layer's planes (keeps the numpy arrays alive)."""
+
+    def __init__(self, layer, K: int):
+        self.arrs = {k: _np(getattr(layer, k)) for k in (
+            "gate_codes", "up_codes", "gate_scales", "up_scales", "gate_global", "up_global",
+            "down_codes", "down_scales", "down_global")}
+        E, I, H2 = self.arrs["gate_codes"].shape
+        self.dims = _Dims(E, H2 * 2, I, K)
+        self.w = _Weights(**{k: v.ctypes.data for k, v in self.arrs.items()})
+
+
+def moe(layer, x, ids, wts, *, K: int, x_scale=None, sample=None, nthreads: int = 0,
+        plant: str | int = 0) -> np.ndarray:
+    """Layer output, FP64 [n][H], for the tokens in `sample` (all when None).
+    x: BF16 [T][H] (torch bf16 or uint16 bits) or int8 [T][H] with x_scale [T]."""
+    b = _Bound(layer, K)
+    xa = _np(x)
+    act_type = 1 if xa.dtype == np.int8 else 0
+    if act_type == 0:
+        xa = xa.view(np.uint16)
+    T = xa.shape[0]
+    xs = _np(x_scale).astype(np.float32) if x_scale is not None else np.zeros(1, np.float32)
+    ia = _np(ids).astype(np.int32)
+    wa = _np(wts).astype(np.float64)
+    samp = None if sample is None else np.ascontiguousarray(np.asarray(sample, np.int32))
+    n = T if samp is None else len(samp)
+    out = np.zeros((n, b.dims.H), np.float64)
+    pl = PLANT[plant] if isinstance(plant, str) else int(plant)
+    rc = lib().orc_moe(C.byref(b.dims), C.byref(b.w), C.c_int32(T), C.c_int32(act_type), _p(xa),
+                       _p(xs), _p(ia), _p(wa), C.c_int32(n),
+                       _p(samp) if samp is not None else None, _p(out), C.c_int32(nthreads),
+                       C.c_int32(pl))
+    assert rc == 0, "oracle rejected its arguments"
+    return out
+
+
+def pair_h(layer, x_row, e: int, *, K: int, x_scale: float = 1.0, plant=0) -> np.ndarray:
+    b = _Bound(layer, K)
+    xa = _np(x_row)
+    act_type = 1 if xa.dtype == np.int8 else 0
+    if act_type == 0:
+        xa = xa.view(np.uint16)
+    h = np.zeros(b.dims.I, np.float64)
+    pl = PLANT[plant] if isinstance(plant, str) else int(plant)
+    lib().orc_pair_h(C.byref(b.dims), C.byref(b.w), act_type, _p(np.ascontiguousarray(xa)),
+                     x_scale, e, _p(h), pl)
+    return h
+
+
+def forward(layer, x, *, K: int, logits=None, ids=None, wts=None, x_scale=None, sample=None,
+            nthreads: int = 0, plant=0):
+    """Route (or take ids/weights as given) and run the layer.
+    -> dict(out, ids, w, counts, offsets, perm, nonfinite)"""
+    E = _np(layer.gate_global).shape[0]
+    if logits is not None:
+        ids, w, bad = route(logits, K)
+    else:
+        ids = _np(ids).astype(np.int32)
+        w = _np(wts).astype(np.float64)
+        bad = 0
+    counts, offsets, perm = sort(ids, E)
+    out = moe(layer, x, ids, w, K=K, x_scale=x_scale, sample=sample, nthreads=nthreads,
+              plant=plant)
+    return dict(out=out, ids=ids, w=w, counts=counts, offsets=offsets, perm=perm, nonfinite=bad)
