@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 MoE layer on B200.
+
+Default workload: the 8192-token prefill chunk of the 512-expert, hidden 2048,
+intermediate 768, top-10 NVFP4 layer with BF16 activations and Zipf(1.1)-skewed
+router logits. One step = the whole layer (routing, sort/permute, gate/up grouped
+GEMM + SwiGLU, down grouped GEMM + weighted combine) over one chunk, inputs
+resident in HBM. Also reported: decode expert GB/s for 1/2/4/8 tokens over 8
+distinct layers, end-to-end throughput through the C ABI with host buffers, the
+dominant kernel's roofline, and the FP64 CPU oracle's throughput.
+
+Multi-GPU: each rank runs its own replica on its own chunk (tokens are
+independent; no data-path collective), value = all ranks' tokens / max time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer prefill tok/s & decode expert GB/s on 1 B200, as % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DECODE_BYTES_PER_EXPERT = None  # set from dims: (3*I*H)/2 codes + (3*I*H)/16 scales
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class Clocks:
+    """Samples nvidia-smi every 100 ms while the timed region runs."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64,
+                     device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle leg
+
+def cpu_oracle_rate(layer_cpu, x, logits, K, n_tokens, x_scale=None):
+    """Tokens/s of the FP64 oracle (as it stands) on a sample of n_tokens tokens."""
+    import oracle
+    sample = np.arange(n_tokens, dtype=np.int32)
+    xs = x[:n_tokens]
+    lg = logits[:n_tokens]
+    t0 = time.perf_counter()
+    oracle.forward(layer_cpu, xs, K=K, logits=lg, x_scale=None if x_scale is None else x_scale[:n_tokens],
+                   sample=sample)
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt
+
+
+# ------------------------------------------------------------------- workloads
+
+def make_prefill(wl_name, dev):
+    wl = synth.CONFIGS[wl_name]
+    d = wl.dims
+    seed = synth.workload_seed(wl)
+    T = wl.tokens[0]
+    layer = synth.make_layer(d, seed, device=dev)
+    logits = synth.make_logits(T, d.E, seed, zipf_s=wl.zipf_s, device=dev)
+    if wl.act == "int8":
+        x, xs = synth.make_x_int8(T, d.H, seed, outliers=wl.outliers, device=dev)
+    else:
+        x, xs = synth.make_x_bf16(T, d.H, seed, outliers=wl.outliers, device=dev), None
+    return wl, layer, logits, x, xs
+
+
+def run_ours(args, ws, rank, local):
+    import nvfp4_mixture_experts_03_b200 as nv
+    dev = torch.device("cuda", local)
+    pk, pk_src = peaks()
+    wl, layer, logits, x, xs = make_prefill(args.workload, dev)
+    d = wl.dims
+    T = x.shape[0]
+    P = T * d.K
+    m = nv.MoELayer.from_layer(layer, top_k=d.K, max_tokens=T)
+    out = torch.empty(T, d.H, dtype=torch.float32, device=dev)
+    ws_buf = m.workspace(T)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        m.forward(x, logits=logits, x_scale=xs, out=out, workspace=ws_buf)
+
+    for _ in range(args.warmup):
+        step()
+    st = m.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    counts = nv.debug_buffers(T, d.E, d.K, dev)
+    m.forward(x, logits=logits, x_scale=xs, out=out, workspace=ws_buf, debug=counts)
+    n_used = int((counts["counts"] > 0).sum().item())
+
+    # phase events per step -> kernel durations over the timed region
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(nv.PHASE_EVENTS)]
+              for _ in range(args.steps)]
+    for evs in evsets:
+        for e in evs:
+            e.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with Clocks(dev.index) as clk:
+        t0.record()
+        for i in range(args.steps):
+            m.set_phase_events(evsets[i])
+            step()
+        t1.record()
+        torch.cuda.synchronize()
+    m.set_phase_events(())
+    barrier(ws)
+    ms = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(ms, ws)
+    phase_ms = np.zeros(nv.PHASE_EVENTS - 1)
+    for evs in evsets:
+        for j in range(nv.PHASE_EVENTS - 1):
+            phase_ms[j] += evs[j].elapsed_time(evs[j + 1])
+    phase_ms /= args.steps
+    st = m.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timed steps")
+
+    value = ws * T * args.steps / (ms_max / 1e3)
+    flops_gu = 2.0 * P * (2 * d.I) * d.H
+    flops_dn = 2.0 * P * d.H * d.I
+    gu_ms = phase_ms[2]
+    achieved = flops_gu / (gu_ms / 1e3) / 1e12
+    peak = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    traffic = profile_traffic("grouped_gemm_gateup")
+    roof = {"kernel": "grouped_gemm_kernel<0> (gate/up + SwiGLU)", "bound": "tensor",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "peak_source": f"{pk_src} bf16_tflops_sustained (F16 operands run at the BF16 rate)",
+            "algorithmic_flops_per_launch": flops_gu}
+    phases = {"routing_ms": round(phase_ms[0], 4), "stage_activations_ms": round(phase_ms[1], 4),
+              "gate_up_ms": round(phase_ms[2], 4), "down_combine_ms": round(phase_ms[3], 4),
+              "down_tflops": round(flops_dn / (phase_ms[3] / 1e3) / 1e12, 1)}
+
+    res = {"metric": METRIC, "value": round(value, 1), "unit": "tok/s", "n_gpus": ws,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f16 (exact NVFP4 dequant, FP32 accumulate)", "data": "synthetic",
+           "config": {"workload": f"{wl.name}: {wl.note}", "tokens_per_rank": T,
+                      "experts_used": n_used,
+                      "l2": "inputs larger than L2 (1.27 GiB of expert planes per layer)",
+                      "parallelism": f"replicas x{ws}"},
+           "roofline": roof, "phases": phases, "clocks": clk.summary(),
+           "gpu_launches": 6 * args.steps}
+
+    # ---- end to end: host buffers, copies inside the timed region
+    if not args.no_e2e:
+        xh = x.cpu().pin_memory()
+        lh = logits.cpu().pin_memory()
+        xsh = xs.cpu().pin_memory() if xs is not None else None
+        oh = torch.empty(T, d.H, dtype=torch.float32).pin_memory()
+        xd, ld_ = torch.empty_like(x), torch.empty_like(logits)
+        xsd = torch.empty_like(xs) if xs is not None else None
+
+        def e2e_step():
+            xd.copy_(xh, non_blocking=True)
+            ld_.copy_(lh, non_blocking=True)
+            if xsd is not None:
+                xsd.copy_(xsh, non_blocking=True)
+            m.forward(xd, logits=ld_, x_scale=xsd, out=out, workspace=ws_buf)
+            oh.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b), ws)
+        h2d = xh.numel() * xh.element_size() + lh.numel() * 4 + (xsh.numel() * 4 if xsh is not None else 0)
+        res["e2e"] = {"value": round(ws * T * args.steps / (e_ms / 1e3), 1), "unit": "tok/s",
+                      "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(oh.numel() * 4)}
+        res["gpu_launches"] += 6 * args.steps
+
+    # ---- decode expert GB/s (8 distinct layers so the L2 never holds the weights)
+    if not args.no_decode:
+        res["decode"] = run_decode(args, dev, pk, pk_src)
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only)
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        layer_cpu = layer.to("cpu")
+        xc, lc = x.cpu(), logits.cpu()
+        xsc = xs.cpu() if xs is not None else None
+        rate, dt = cpu_oracle_rate(layer_cpu, xc, lc, d.K, 8, xsc)       # calibrate
+        n = int(min(T, max(8, rate * args.cpu_seconds)))
+        rate, dt = cpu_oracle_rate(layer_cpu, xc, lc, d.K, n, xsc)
+        res["cpu_baseline"] = {"value": round(rate, 3), "unit": "tok/s", "cores": os.cpu_count(),
+                               "kind": "oracle",
+                               "sample": f"first {n} of the {T} tokens of the same chunk, FP64, "
+                                         f"{dt:.1f} s wall"}
+    m.close()
+    return res
+
+
+def run_decode(args, dev, pk, pk_src):
+    import nvfp4_mixture_experts_03_b200 as nv
+    wl = synth.CONFIGS["decode"]
+    d = wl.dims
+    nl = args.decode_layers
+    per_expert = (3 * d.I * d.H) // 2 + (3 * d.I * d.H) // 16
+    layers = [synth.make_layer(d, synth.workload_seed(wl, l), device=dev) for l in range(nl)]
+    models = [nv.MoELayer.from_layer(L, top_k=d.K, max_tokens=8) for L in layers]
+    out = {}
+    for T in wl.tokens:
+        xs = [synth.make_x_bf16(T, d.H, synth.workload_seed(wl, l) + 17 * T, outliers=True, device=dev)
+              for l in range(nl)]
+        lg = [synth.make_logits(T, d.E, synth.workload_seed(wl, l) + 17 * T, zipf_s=wl.zipf_s,
+                                device=dev) for l in range(nl)]
+        outs = [torch.empty(T, d.H, dtype=torch.float32, device=dev) for _ in range(nl)]
+        uniq = 0
+        for l in range(nl):
+            dbg = nv.debug_buffers(T, d.E, d.K, dev)
+            models[l].forward(xs[l], logits=lg[l], out=outs[l], debug=dbg)
+            uniq += int((dbg["counts"] > 0).sum().item())
+        ws_bufs = [mm.workspace(T) for mm in models]
+
+        def step():
+            for l in range(nl):
+                models[l].forward(xs[l], logits=lg[l], out=outs[l], workspace=ws_bufs[l])
+
+        for _ in range(args.warmup):
+            step()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nv.PHASE_EVENTS)]
+               for _ in range(nl * args.steps)]
+        for es in evs:
+            for e in es:
+                e.record()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        k = 0
+        for _ in range(args.steps):
+            for l in range(nl):
+                models[l].set_phase_events(evs[k])
+                k += 1
+                models[l].forward(xs[l], logits=lg[l], out=outs[l], workspace=ws_bufs[l])
+        b.record()
+        torch.cuda.synchronize()
+        for mm in models:
+            mm.set_phase_events(())
+        ms = a.elapsed_time(b) / args.steps
+        kern_ms = sum(es[2].elapsed_time(es[4]) for es in evs) / args.steps
+        nbytes = uniq * per_expert
+        gbs = nbytes / (ms / 1e3) / 1e9
+        kgbs = nbytes / (kern_ms / 1e3) / 1e9
+        out[f"T{T}"] = {"layers": nl, "unique_experts": uniq, "bytes": nbytes,
+                        "layer_us": round(ms * 1e3 / nl, 2), "GBps_layer": round(gbs, 1),
+                        "GBps_expert_kernels": round(kgbs, 1),
+                        "frac_layer": round(gbs / pk["hbm_gbs"], 4),
+                        "frac_expert_kernels": round(kgbs / pk["hbm_gbs"], 4)}
+    out["peak"] = {"hbm_gbs": pk["hbm_gbs"], "source": pk_src}
+    for mm in models:
+        mm.close()
+    return out
+
+
+def profile_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    import hashlib
+    rec = json.load(open(p)).get(kernel_key)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["dram_bytes_per_launch"] if h == rec["source_sha256_16"] else None
+
+
+# --------------------------------------------------------- reference (oracle) arm
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return None
+    wl = synth.CONFIGS[args.workload]
+    d = wl.dims
+    seed = synth.workload_seed(wl)
+    T = wl.tokens[0]
+    n = args.ref_tokens
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"   # same draw as the GPU arm
+    layer = synth.make_layer(d, seed, device=gen_dev).to("cpu")
+    logits = synth.make_logits(T, d.E, seed, zipf_s=wl.zipf_s, device=gen_dev).cpu()
+    if wl.act == "int8":
+        x, xs = synth.make_x_int8(T, d.H, seed, outliers=wl.outliers, device=gen_dev)
+        x, xs = x.cpu(), xs.cpu()
+    else:
+        x, xs = synth.make_x_bf16(T, d.H, seed, outliers=wl.outliers, device=gen_dev).cpu(), None
+    for _ in range(args.warmup):
+        cpu_oracle_rate(layer, x, logits, d.K, n, xs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cpu_oracle_rate(layer, x, logits, d.K, n, xs)
+    dt = time.perf_counter() - t0
+    v = n * args.steps / dt
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tok/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3 / args.steps, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: {wl.note}", "tokens_per_step": n},
+            "cpu_baseline": {"value": round(v, 3), "unit": "tok/s", "cores": os.cpu_count(),
+                             "kind": "oracle",
+                             "sample": f"first {n} tokens of the {T}-token chunk per step"},
+            "e2e": {"value": round(v, 3), "unit": "tok/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill8k", choices=["prefill8k", "w4a8_32k"])
+    ap.add_argument("--decode-layers", type=int, default=8)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-tokens", type=int, default=16)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    ws, rank, local = dist_setup()
+    if args.impl == "reference":
+        res = run_reference(args, ws, rank)
+    else:
+        res = run_ours(args, ws, rank, local)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

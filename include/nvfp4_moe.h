@@ -67,6 +67,12 @@ extern "C" {
 
 #define NVFP4_MOE_ABI_VERSION 1
 
+#if defined(__GNUC__)
+#define NVFP4_MOE_API __attribute__((visibility("default")))
+#else
+#define NVFP4_MOE_API
+#endif
+
 /* Largest top-k the kernels support, and the largest T the decode path takes. */
 #define NVFP4_MOE_MAX_TOPK 16
 #define NVFP4_MOE_DECODE_MAX_T 8
@@ -117,8 +123,12 @@ typedef struct {
 } nvfp4_moe_weights;
 
 typedef enum {
-    NVFP4_MOE_ACT_BF16 = 0, /* act is [T][H] bf16                                */
-    NVFP4_MOE_ACT_INT8 = 1  /* act is [T][H] int8 q, x = q * act_scale[t] (f32) */
+    NVFP4_MOE_ACT_BF16 = 0, /* act is [T][H] bf16                                 */
+    NVFP4_MOE_ACT_INT8 = 1, /* act is [T][H] int8 q, x = q * act_scale[t] (f32)  */
+    NVFP4_MOE_ACT_F32 = 2   /* act is [T][H] f32 (a residual stream); the layer's
+                               input is its round-to-nearest-even BF16 value.
+                               act may equal out with NVFP4_MOE_OUT_F32_ADD:
+                               x <- x + layer(bf16(x)), one stacked-layer step.  */
 } nvfp4_moe_act;
 
 typedef enum {
@@ -158,32 +168,43 @@ typedef struct {
  * allocates the handle and its 64-byte device status block on the current device.
  * On failure *out is set to NULL and nothing stays allocated. Requires an sm_100
  * device to be current. */
-int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
+NVFP4_MOE_API int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
                      const nvfp4_moe_weights *weights);
 
 /* Bytes of workspace a forward call with T tokens needs (256-byte aligned start
  * required). Returns 0 for a NULL handle or T outside [0, max_tokens]. */
-size_t nvfp4_moe_workspace_bytes(const nvfp4_moe_t *h, int32_t T);
+NVFP4_MOE_API size_t nvfp4_moe_workspace_bytes(const nvfp4_moe_t *h, int32_t T);
 
 /* Enqueues the whole layer on `stream` (a cudaStream_t; NULL = legacy default
  * stream). Asynchronous: never synchronises and never reads device memory back.
  * The workspace must not be used by another call until this one has finished
  * on the GPU. */
-int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *workspace,
+NVFP4_MOE_API int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *workspace,
                       size_t workspace_bytes, void *stream);
 
 /* Synchronises `stream`, returns the first device-side error latched since the
  * last call (0 if none) and clears it. */
-int nvfp4_moe_get_status(nvfp4_moe_t *h, void *stream);
+NVFP4_MOE_API int nvfp4_moe_get_status(nvfp4_moe_t *h, void *stream);
+
+/* Phase timing (optional): when n_events == NVFP4_MOE_PHASE_EVENTS and events
+ * holds that many cudaEvent_t handles (created by the caller on the handle's
+ * device), every later forward records event i on its stream at these phase
+ * boundaries: 0 start, 1 routing done, 2 activation staging done, 3 gate/up +
+ * SwiGLU done, 4 down + combine done. (Decode calls stage activations inside
+ * routing, so events 1 and 2 coincide.) n_events == 0 turns it off. The handle
+ * borrows the events; returns INVALID_ARG for any other n_events. This mirrors
+ * per-phase accounting of a layer's time; it adds four event records per call. */
+#define NVFP4_MOE_PHASE_EVENTS 5
+NVFP4_MOE_API int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events, int32_t n_events);
 
 /* Frees the handle and its status block. Never touches the borrowed weights. */
-void nvfp4_moe_destroy(nvfp4_moe_t *h);
+NVFP4_MOE_API void nvfp4_moe_destroy(nvfp4_moe_t *h);
 
 /* Static string for a status code. */
-const char *nvfp4_moe_strerror(int status);
+NVFP4_MOE_API const char *nvfp4_moe_strerror(int status);
 
 /* ABI version compiled into the library (NVFP4_MOE_ABI_VERSION). */
-int nvfp4_moe_abi_version(void);
+NVFP4_MOE_API int nvfp4_moe_abi_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,302 @@
+// Device helpers shared by the layer's kernels (sm_100a only): status latching,
+// bounded mbarrier waits, TMA loads, tcgen05 (TMEM alloc / MMA / commit / load),
+// NVFP4 conversions, and the workspace / launch-parameter layout.
+#pragma once
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "nvfp4_moe.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "this library targets sm_100a only"
+#endif
+
+namespace nvmoe {
+
+// ---------------------------------------------------------------- constants
+constexpr int kChunkTokens = 64;       // tokens per routing CTA (two 32-bit token masks)
+constexpr int kBN = 256;               // max tokens per grouped-GEMM tile (MMA N)
+constexpr int kBK = 64;                // K elements per pipeline stage (one 128B swizzle row)
+constexpr int kGuRows = 64;            // intermediate rows per gate/up tile (64 gate + 64 up)
+constexpr int kDnRows = 128;           // hidden rows per down tile
+constexpr int kStages = 4;             // smem pipeline depth of the grouped GEMM
+
+// Device status block layout (int32 words).
+enum : int { kStatusCode = 0, kStatusDetail = 1, kStatusWords = 16 };
+
+// Per-call routing/tile counters kept in the workspace (int32 words).
+enum : int { kCntTilesGu = 0, kCntTilesDn = 1, kCntUniq = 2, kCntWords = 64 };
+
+struct Tile {  // one grouped-GEMM tile
+    int32_t expert;   // expert id
+    int32_t m0;       // first output row (gate/up: intermediate index; down: hidden index)
+    int32_t pos0;     // first pair position (rows of the permuted activations / h)
+    int32_t ntok;     // valid pairs in this tile (1..kBN)
+};
+
+// Everything a forward call's kernels read, passed by value.
+struct Params {
+    int32_t T, E, H, I, K;
+    int32_t act_type;          // nvfp4_moe_act, plus kActF32 below
+    int32_t out_add;           // 1: out += layer(x)
+    const void *act;
+    const float *act_scale;
+    const float *logits;       // may be null
+    const int32_t *in_ids;     // precomputed routing when logits == null
+    const float *in_w;
+    float *out;
+    // weights
+    const uint8_t *gate_codes, *up_codes, *gate_scales, *up_scales;
+    const float *gate_global, *up_global;
+    const uint8_t *down_codes, *down_scales;
+    const float *down_global;
+    // workspace regions
+    int32_t *cnt;              // kCntWords counters
+    int32_t *ids;              // [P]
+    float *wts;                // [P]
+    int32_t *hist;             // [E][nch]
+    int32_t *cbase;            // [E][nch]
+    int32_t *counts;           // [E]
+    int32_t *offsets;          // [E+1]
+    int32_t *perm;             // [P] pair index at each position
+    int32_t *inv;              // [P] position of each pair
+    int32_t *ptok;             // [P] token at each position
+    float *pw;                 // [P] routing weight at each position
+    float *ps;                 // [P] activation scale at each position (prefill)
+    float *xscale;             // [T] activation scale per token
+    Tile *tiles_gu, *tiles_dn;
+    int32_t *uniq;             // [<=P] decode: unique experts ascending
+    int32_t *upos;             // [<=P][8] decode: position of (unique expert, token) or -1
+    __half *xh;                // prefill: [P][H] permuted activations; decode: [T][H]
+    __half *h;                 // [P][I]
+    int32_t *status;           // device status block
+    // optional debug copies
+    int32_t *dbg_ids;
+    float *dbg_w;
+    int32_t *dbg_counts, *dbg_offsets, *dbg_perm;
+    int32_t nch;               // routing chunks
+    int32_t max_tiles_gu, max_tiles_dn;
+};
+
+constexpr int kActF32 = 2;     // internal: act is FP32, rounded to BF16 first
+
+__host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------------ status
+__device__ inline void latch_status(int32_t *status, int code, int detail) {
+    if (atomicCAS(&status[kStatusCode], 0, code) == 0) status[kStatusDetail] = detail;
+}
+
+// --------------------------------------------------------------- utilities
+__device__ inline uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ inline uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ inline void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ inline void mbar_arrive(uint64_t *bar) {
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+__device__ inline void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile(
+        "{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}" ::"r"(
+            smem_u32(bar)),
+        "r"(bytes)
+        : "memory");
+}
+__device__ inline bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait: gives up after `limit_ns` of wall time (or when *abort is set by
+// another thread), latching NVFP4_MOE_ERR_TIMEOUT. Returns false on give-up.
+__device__ inline bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                 int32_t *status, int where, uint64_t limit_ns = 2000000000ull) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    uint32_t spins = 0;
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((++spins & 63) == 0) {
+            if (*abort) return false;
+            if (globaltimer() - t0 > limit_ns) {
+                *abort = 1;
+                latch_status(status, NVFP4_MOE_ERR_TIMEOUT, where);
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded wait used when draining after a give-up: ignores the abort flag, never
+// latches a status, returns false after `limit_ns`.
+__device__ inline bool mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > limit_ns) return false;
+    return true;
+}
+
+__device__ inline void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ inline void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// --------------------------------------------------------------------- TMA
+__device__ inline void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x,
+                                   int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ inline void tma_prefetch_desc(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
+}
+
+// ----------------------------------------------------------------- tcgen05
+__device__ inline void tmem_alloc(uint32_t *slot_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(slot_smem)),
+                 "r"(ncols));
+}
+__device__ inline void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+}
+__device__ inline void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+__device__ inline void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ inline void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem desc] x B[smem desc]^T, kind::f16 (both operands F16), one CTA.
+__device__ inline void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                  uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// Arrives on `bar` once every tcgen05.mma issued so far by this thread has completed.
+__device__ inline void tc_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+// 32 lanes x 32 consecutive 32-bit columns: this thread gets its lane's 32 columns.
+__device__ inline void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ inline void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major operand tile in the 128-byte swizzle
+// layout (rows of 128 B, 8-row groups 1024 B apart). Start address in 16-B units.
+__device__ inline uint64_t smem_desc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);            // start address
+    d |= (uint64_t)1 << 16;                             // leading byte offset (unused for SW128 K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;                   // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;                             // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;                             // layout: 128-byte swizzle
+    return d;
+}
+// Instruction descriptor, kind::f16: F16 x F16 -> F32, both K-major, M x N.
+__host__ __device__ inline uint32_t idesc_f16(int M, int N) {
+    return (1u << 4)                      // D format F32
+           | (0u << 7) | (0u << 10)       // A, B format F16
+           | ((uint32_t)(N >> 3) << 17)   // N / 8
+           | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// ------------------------------------------------------- NVFP4 conversions
+// Four E2M1 code bytes -> four f16x2 (low nibble -> low half: element 2c first).
+__device__ inline void e2m1x8_to_f16(uint32_t c, uint32_t &o0, uint32_t &o1, uint32_t &o2,
+                                     uint32_t &o3) {
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"
+        " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+        " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+        : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
+        : "r"(c));
+}
+// One E4M3 scale byte -> f16x2 with the scale in both halves (exact: E4M3 is a
+// subset of F16).
+__device__ inline uint32_t e4m3_to_f16x2_bcast(uint32_t s) {
+    uint32_t o;
+    const uint16_t two = (uint16_t)((s & 0xFF) | ((s & 0xFF) << 8));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(o) : "h"(two));
+    return o;
+}
+__device__ inline uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// ----------------------------------------------------------------- mma.sync
+// D[16x8] += A[16x16] (row) x B[16x8] (col), F16 inputs, F32 accumulate.
+__device__ inline void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                 uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ inline float silu(float z) { return z / (1.0f + __expf(-z)); }
+
+// Per-token power-of-two factor 2^k with amax * 2^k in [2^14, 2^15): every BF16
+// value within 2^28 of the token's amax is exact in F16 after the shift.
+__device__ inline int pow2_shift_for(float amax) {
+    if (!(amax > 0.0f) || !isfinite(amax)) return 0;
+    int e;
+    frexpf(amax, &e);           // amax = m * 2^e, m in [0.5, 1)
+    int k = 15 - e;             // amax * 2^k in [2^14, 2^15)
+    return k < -120 ? -120 : (k > 120 ? 120 : k);   // keep 2^-k a normal FP32
+}
+
+// ------------------------------------------------------------ kernel decls
+void launch_route_large(const Params &p, cudaStream_t s);
+void launch_route_small(const Params &p, cudaStream_t s);
+void launch_prep_prefill(const Params &p, cudaStream_t s);
+void launch_decode_gateup(const Params &p, cudaStream_t s);
+void launch_decode_down(const Params &p, cudaStream_t s);
+// mode 0: gate/up + SwiGLU over map = F16 activations [P][H]; mode 1: down + combine over map = h [P][I]
+void launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &map, int num_sms,
+                         cudaStream_t s);
+cudaError_t prefill_init();   // per device: opt the GEMM kernels into their shared memory
+
+}  // namespace nvmoe

@@ -1,0 +1,326 @@
+// Host side of the C ABI declared in include/nvfp4_moe.h: argument validation
+// (all of it before any allocation or launch), the workspace layout, TMA tensor
+// maps for the grouped GEMMs, and the launch sequence of one forward call.
+//
+// Conventions follow the pages' readers ("#1858 ... strata-safetensors",
+// "Proposed contribution": bounded caller-owned buffers; "TensorFold PR #906",
+// first post: complete validation before allocation, nothing left allocated on
+// failure): the caller owns every buffer, including the workspace.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "common.cuh"
+
+using namespace nvmoe;
+
+struct nvfp4_moe {
+    nvfp4_moe_dims d;
+    nvfp4_moe_weights w;
+    int device;
+    int num_sms;
+    int32_t *status;  // kStatusWords ints on the device
+    cudaEvent_t phase[NVFP4_MOE_PHASE_EVENTS];
+    bool phase_on;
+};
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2D F16 tensor [rows][cols], box 64 x 64, 128-byte swizzle, zero fill outside.
+bool make_map_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, 64};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
+
+struct WsLayout {
+    size_t cnt, ids, wts, hist, cbase, counts, offsets, perm, inv, ptok, pw, ps, xscale, tiles_gu,
+        tiles_dn, uniq, upos, xh, h, total;
+    int nch, max_gu, max_dn;
+};
+
+WsLayout layout(const nvfp4_moe_dims &d, int T) {
+    WsLayout L{};
+    const size_t P = (size_t)T * d.top_k;
+    const int E = d.n_experts;
+    L.nch = cdiv(T > 0 ? T : 1, kChunkTokens);
+    const bool decode = T <= NVFP4_MOE_DECODE_MAX_T;
+    const size_t ntile_n = P / kBN + (size_t)(E < (int)P ? E : (int)P) + 1;
+    L.max_gu = decode ? 0 : (int)(ntile_n * (d.inter / kGuRows));
+    L.max_dn = decode ? 0 : (int)(ntile_n * (d.hidden / kDnRows));
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = a256(o + bytes);
+        return at;
+    };
+    L.cnt = take(kCntWords * 4);
+    L.ids = take(P * 4);
+    L.wts = take(P * 4);
+    L.hist = take(decode ? 0 : (size_t)E * L.nch * 4);
+    L.cbase = take(decode ? 0 : (size_t)E * L.nch * 4);
+    L.counts = take((size_t)E * 4);
+    L.offsets = take((size_t)(E + 1) * 4);
+    L.perm = take(P * 4);
+    L.inv = take(P * 4);
+    L.ptok = take(P * 4);
+    L.pw = take(P * 4);
+    L.ps = take(P * 4);
+    L.xscale = take((size_t)T * 4);
+    L.tiles_gu = take((size_t)L.max_gu * sizeof(Tile));
+    L.tiles_dn = take((size_t)L.max_dn * sizeof(Tile));
+    L.uniq = take(decode ? P * 4 : 0);
+    L.upos = take(decode ? P * NVFP4_MOE_DECODE_MAX_T * 4 : 0);
+    L.xh = take((decode ? (size_t)T : P) * d.hidden * 2);
+    L.h = take(P * d.inter * 2);
+    L.total = o;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nvfp4_moe_abi_version(void) { return NVFP4_MOE_ABI_VERSION; }
+
+const char *nvfp4_moe_strerror(int s) {
+    switch (s) {
+        case NVFP4_MOE_OK: return "ok";
+        case NVFP4_MOE_ERR_INVALID_ARG: return "invalid argument";
+        case NVFP4_MOE_ERR_UNSUPPORTED_DIMS: return "unsupported dimensions";
+        case NVFP4_MOE_ERR_MISALIGNED: return "misaligned pointer";
+        case NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case NVFP4_MOE_ERR_CUDA: return "CUDA error";
+        case NVFP4_MOE_ERR_BAD_ROUTING: return "routing id out of range or repeated";
+        case NVFP4_MOE_ERR_NONFINITE: return "non-finite routing logit";
+        case NVFP4_MOE_ERR_TIMEOUT: return "device wait timed out";
+        case NVFP4_MOE_ERR_NO_DEVICE: return "no sm_100 device";
+        default: return "unknown status";
+    }
+}
+
+int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
+                     const nvfp4_moe_weights *w) {
+    if (!out) return NVFP4_MOE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!dims || !w) return NVFP4_MOE_ERR_INVALID_ARG;
+    const nvfp4_moe_dims d = *dims;
+    if (d.hidden <= 0 || d.inter <= 0 || d.n_experts <= 0 || d.top_k <= 0 || d.max_tokens < 0)
+        return NVFP4_MOE_ERR_INVALID_ARG;
+    if (d.hidden % 128 || d.inter % 128 || d.top_k > d.n_experts ||
+        d.top_k > NVFP4_MOE_MAX_TOPK || d.n_experts > 1024)
+        return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
+    if ((int64_t)d.max_tokens * d.top_k > (1 << 30)) return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
+    const void *planes[] = {w->gate_codes, w->up_codes, w->gate_scales, w->up_scales,
+                            w->down_codes, w->down_scales};
+    const void *globals[] = {w->gate_global, w->up_global, w->down_global};
+    for (const void *p : planes)
+        if (!p) return NVFP4_MOE_ERR_INVALID_ARG;
+    for (const void *p : globals)
+        if (!p) return NVFP4_MOE_ERR_INVALID_ARG;
+    for (const void *p : planes)
+        if (!al16(p)) return NVFP4_MOE_ERR_MISALIGNED;
+    for (const void *p : globals)
+        if (!al4(p)) return NVFP4_MOE_ERR_MISALIGNED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_MOE_ERR_NO_DEVICE;
+    int major = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (major != 10) return NVFP4_MOE_ERR_NO_DEVICE;
+    if (prefill_init() != cudaSuccess || !encode_fn()) return NVFP4_MOE_ERR_CUDA;
+    nvfp4_moe *h = new (std::nothrow) nvfp4_moe;
+    if (!h) return NVFP4_MOE_ERR_CUDA;
+    h->d = d;
+    h->w = *w;
+    h->device = dev;
+    h->num_sms = sms;
+    h->status = nullptr;
+    h->phase_on = false;
+    if (cudaMalloc(&h->status, kStatusWords * sizeof(int32_t)) != cudaSuccess ||
+        cudaMemset(h->status, 0, kStatusWords * sizeof(int32_t)) != cudaSuccess) {
+        if (h->status) cudaFree(h->status);
+        delete h;
+        return NVFP4_MOE_ERR_CUDA;
+    }
+    *out = h;
+    return NVFP4_MOE_OK;
+}
+
+size_t nvfp4_moe_workspace_bytes(const nvfp4_moe_t *h, int32_t T) {
+    if (!h || T < 0 || T > h->d.max_tokens) return 0;
+    return layout(h->d, T).total;
+}
+
+int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t ws_bytes,
+                      void *stream) {
+    if (!h || !io) return NVFP4_MOE_ERR_INVALID_ARG;
+    const nvfp4_moe_dims &d = h->d;
+    const int T = io->T;
+    if (T < 0 || T > d.max_tokens) return NVFP4_MOE_ERR_INVALID_ARG;
+    if (io->act_type != NVFP4_MOE_ACT_BF16 && io->act_type != NVFP4_MOE_ACT_INT8 &&
+        io->act_type != NVFP4_MOE_ACT_F32)
+        return NVFP4_MOE_ERR_INVALID_ARG;
+    if (io->out_type != NVFP4_MOE_OUT_F32 && io->out_type != NVFP4_MOE_OUT_F32_ADD)
+        return NVFP4_MOE_ERR_INVALID_ARG;
+    if (T == 0) return NVFP4_MOE_OK;
+    if (!io->act || !io->out) return NVFP4_MOE_ERR_INVALID_ARG;
+    if (io->act_type == NVFP4_MOE_ACT_INT8 && !io->act_scale) return NVFP4_MOE_ERR_INVALID_ARG;
+    if (!io->router_logits && (!io->topk_ids || !io->topk_weights)) return NVFP4_MOE_ERR_INVALID_ARG;
+    if (io->act == io->out && io->out_type != NVFP4_MOE_OUT_F32_ADD) return NVFP4_MOE_ERR_INVALID_ARG;
+    if (!al16(io->act) || !al16(io->out) || (io->router_logits && !al16(io->router_logits)) ||
+        (io->act_scale && !al4(io->act_scale)) || (io->topk_ids && !al4(io->topk_ids)) ||
+        (io->topk_weights && !al4(io->topk_weights)))
+        return NVFP4_MOE_ERR_MISALIGNED;
+    const WsLayout L = layout(d, T);
+    if (!ws || ws_bytes < L.total) return NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (reinterpret_cast<uintptr_t>(ws) & 255) return NVFP4_MOE_ERR_MISALIGNED;
+
+    uint8_t *b = static_cast<uint8_t *>(ws);
+    Params p{};
+    p.T = T;
+    p.E = d.n_experts;
+    p.H = d.hidden;
+    p.I = d.inter;
+    p.K = d.top_k;
+    p.act_type = io->act_type;
+    p.out_add = io->out_type == NVFP4_MOE_OUT_F32_ADD;
+    p.act = io->act;
+    p.act_scale = io->act_scale;
+    p.logits = io->router_logits;
+    p.in_ids = io->topk_ids;
+    p.in_w = io->topk_weights;
+    p.out = io->out;
+    p.gate_codes = h->w.gate_codes;
+    p.up_codes = h->w.up_codes;
+    p.gate_scales = h->w.gate_scales;
+    p.up_scales = h->w.up_scales;
+    p.gate_global = h->w.gate_global;
+    p.up_global = h->w.up_global;
+    p.down_codes = h->w.down_codes;
+    p.down_scales = h->w.down_scales;
+    p.down_global = h->w.down_global;
+    p.cnt = reinterpret_cast<int32_t *>(b + L.cnt);
+    p.ids = reinterpret_cast<int32_t *>(b + L.ids);
+    p.wts = reinterpret_cast<float *>(b + L.wts);
+    p.hist = reinterpret_cast<int32_t *>(b + L.hist);
+    p.cbase = reinterpret_cast<int32_t *>(b + L.cbase);
+    p.counts = reinterpret_cast<int32_t *>(b + L.counts);
+    p.offsets = reinterpret_cast<int32_t *>(b + L.offsets);
+    p.perm = reinterpret_cast<int32_t *>(b + L.perm);
+    p.inv = reinterpret_cast<int32_t *>(b + L.inv);
+    p.ptok = reinterpret_cast<int32_t *>(b + L.ptok);
+    p.pw = reinterpret_cast<float *>(b + L.pw);
+    p.ps = reinterpret_cast<float *>(b + L.ps);
+    p.xscale = reinterpret_cast<float *>(b + L.xscale);
+    p.tiles_gu = reinterpret_cast<Tile *>(b + L.tiles_gu);
+    p.tiles_dn = reinterpret_cast<Tile *>(b + L.tiles_dn);
+    p.uniq = reinterpret_cast<int32_t *>(b + L.uniq);
+    p.upos = reinterpret_cast<int32_t *>(b + L.upos);
+    p.xh = reinterpret_cast<__half *>(b + L.xh);
+    p.h = reinterpret_cast<__half *>(b + L.h);
+    p.status = h->status;
+    p.dbg_ids = io->dbg_ids;
+    p.dbg_w = io->dbg_w;
+    p.dbg_counts = io->dbg_counts;
+    p.dbg_offsets = io->dbg_offsets;
+    p.dbg_perm = io->dbg_perm;
+    p.nch = L.nch;
+    p.max_tiles_gu = L.max_gu;
+    p.max_tiles_dn = L.max_dn;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto mark = [&](int i) {
+        if (h->phase_on) cudaEventRecord(h->phase[i], s);
+    };
+    if (T <= NVFP4_MOE_DECODE_MAX_T) {
+        mark(0);
+        launch_route_small(p, s);
+        mark(1);
+        mark(2);
+        launch_decode_gateup(p, s);
+        mark(3);
+        launch_decode_down(p, s);
+        mark(4);
+    } else {
+        const int64_t P = (int64_t)T * d.top_k;
+        CUtensorMap map_xh, map_h;
+        if (!make_map_f16(&map_xh, p.xh, P, d.hidden) || !make_map_f16(&map_h, p.h, P, d.inter))
+            return NVFP4_MOE_ERR_CUDA;
+        mark(0);
+        launch_route_large(p, s);
+        mark(1);
+        launch_prep_prefill(p, s);
+        mark(2);
+        launch_prefill_gemm(0, p, map_xh, h->num_sms, s);
+        mark(3);
+        launch_prefill_gemm(1, p, map_h, h->num_sms, s);
+        mark(4);
+    }
+    return cudaGetLastError() == cudaSuccess ? NVFP4_MOE_OK : NVFP4_MOE_ERR_CUDA;
+}
+
+int nvfp4_moe_get_status(nvfp4_moe_t *h, void *stream) {
+    if (!h) return NVFP4_MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t st[kStatusWords];
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
+    if (cudaMemcpy(st, h->status, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return NVFP4_MOE_ERR_CUDA;
+    if (cudaMemset(h->status, 0, sizeof(st)) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
+    return st[kStatusCode];
+}
+
+int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events, int32_t n_events) {
+    if (!h) return NVFP4_MOE_ERR_INVALID_ARG;
+    if (n_events == 0) {
+        h->phase_on = false;
+        return NVFP4_MOE_OK;
+    }
+    if (n_events != NVFP4_MOE_PHASE_EVENTS || !events) return NVFP4_MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < NVFP4_MOE_PHASE_EVENTS; i++)
+        if (!events[i]) return NVFP4_MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < NVFP4_MOE_PHASE_EVENTS; i++) h->phase[i] = static_cast<cudaEvent_t>(events[i]);
+    h->phase_on = true;
+    return NVFP4_MOE_OK;
+}
+
+void nvfp4_moe_destroy(nvfp4_moe_t *h) {
+    if (!h) return;
+    if (h->status) cudaFree(h->status);
+    delete h;
+}
+
+}  // extern "C"

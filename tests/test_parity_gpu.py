@@ -1,0 +1,168 @@
+"""GPU parity: the CUDA layer, called through the C ABI, against the FP64 oracle
+on the same seeded inputs. Routing ids, counts, offsets and the permutation must
+match bit for bit; routing weights to FP32 rounding; the layer output within
+normalised L2 <= 2e-3 and max elementwise relative error <= 1e-2."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import assert_close, check_routing, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _case(dims, T, seed, *, zipf=None, act="bf16", outliers=False):
+    layer = synth.make_layer(dims, seed)
+    logits = synth.make_logits(T, dims.E, seed, zipf_s=zipf)
+    if act == "int8":
+        x, xs = synth.make_x_int8(T, dims.H, seed, outliers=outliers)
+    else:
+        x, xs = synth.make_x_bf16(T, dims.H, seed, outliers=outliers), None
+    return layer, logits, x, xs
+
+
+def _run_both(layer, logits, x, xs, K, **kw):
+    ref = oracle.forward(layer, x, K=K, logits=logits, x_scale=xs)
+    lg = layer.to(DEV)
+    out, dbg, st = run_gpu(lg, x.to(DEV), K=K, logits=logits.to(DEV),
+                           x_scale=None if xs is None else xs.to(DEV), **kw)
+    return ref, out, dbg, st
+
+
+# T <= 8 takes the decode (GEMV) path, larger T the grouped-GEMM path.
+@pytest.mark.parametrize("T", [1, 3, 8, 9, 64, 200])
+def test_tiny_layer_bf16(T):
+    dims = synth.TINY
+    layer, logits, x, xs = _case(dims, T, seed=synth.BASE_SEED + T)
+    ref, out, dbg, st = _run_both(layer, logits, x, xs, dims.K)
+    assert st == 0
+    check_routing(dbg, ref, T, dims.K)
+    assert_close(out, ref["out"], f"tiny T={T}")
+
+
+@pytest.mark.parametrize("T", [2, 64])
+def test_tiny_layer_int8(T):
+    dims = synth.TINY
+    layer, logits, x, xs = _case(dims, T, seed=700 + T, act="int8", outliers=True)
+    ref, out, dbg, st = _run_both(layer, logits, x, xs, dims.K)
+    assert st == 0
+    check_routing(dbg, ref, T, dims.K)
+    assert_close(out, ref["out"], f"tiny int8 T={T}")
+
+
+@pytest.mark.parametrize("T", [5, 300])
+def test_precomputed_routing(T):
+    dims = synth.LayerDims(E=16, H=256, I=256, K=4)
+    layer = synth.make_layer(dims, seed=31)
+    x = synth.make_x_bf16(T, dims.H, seed=32)
+    ids, w = synth.make_topk(T, dims.E, dims.K, seed=33)
+    ref = oracle.forward(layer, x, K=dims.K, ids=ids, wts=w)
+    out, dbg, st = run_gpu(layer.to(DEV), x.to(DEV), K=dims.K, ids=ids.to(DEV), wts=w.to(DEV))
+    assert st == 0
+    assert np.array_equal(dbg["perm"].numpy(), ref["perm"])
+    assert np.array_equal(dbg["counts"].numpy(), ref["counts"])
+    assert_close(out, ref["out"], "precomputed routing")
+
+
+@pytest.mark.parametrize("T", [4, 700])
+def test_medium_skewed_multi_tile(T):
+    """Zipf-skewed routing: a hot expert spans several 256-pair tiles, a ragged
+    last tile, and several experts stay empty."""
+    dims = synth.LayerDims(E=64, H=512, I=384, K=6)
+    layer, logits, x, xs = _case(dims, T, seed=41, zipf=1.1, outliers=True)
+    ref, out, dbg, st = _run_both(layer, logits, x, xs, dims.K)
+    assert st == 0
+    check_routing(dbg, ref, T, dims.K)
+    if T > 8:
+        assert ref["counts"].max() > 256 and (ref["counts"] == 0).any()
+    assert_close(out, ref["out"], f"medium T={T}")
+
+
+def test_one_expert_takes_every_token_and_k_equals_e():
+    dims = synth.LayerDims(E=8, H=256, I=128, K=8)
+    T = 40
+    layer, logits, x, xs = _case(dims, T, seed=51)
+    ref, out, dbg, st = _run_both(layer, logits, x, xs, dims.K)
+    assert st == 0 and (ref["counts"] == T).all()
+    check_routing(dbg, ref, T, dims.K)
+    assert_close(out, ref["out"], "K = E")
+
+
+def test_k1_single_hot_expert():
+    dims = synth.LayerDims(E=8, H=256, I=128, K=1)
+    T = 270
+    layer, logits, x, xs = _case(dims, T, seed=52)
+    logits[:, 5] += 100.0
+    ref, out, dbg, st = _run_both(layer, logits, x, xs, 1)
+    assert st == 0 and ref["counts"][5] == T
+    check_routing(dbg, ref, T, 1)
+    assert_close(out, ref["out"], "K = 1, one expert")
+
+
+def test_residual_stream_accumulate():
+    """x <- x + layer(bf16(x)) in place (act == out, FP32 residual)."""
+    dims = synth.TINY
+    T = 48
+    layer, logits, _, _ = _case(dims, T, seed=53)
+    x32 = synth.make_x_f32(T, dims.H, seed=54, outliers=False)
+    xb = x32.to(torch.bfloat16)
+    ref = oracle.forward(layer, xb, K=dims.K, logits=logits)
+    xg = x32.to(DEV).contiguous()
+    out, dbg, st = run_gpu(layer.to(DEV), xg, K=dims.K, logits=logits.to(DEV), out=xg,
+                           accumulate=True)
+    assert st == 0
+    assert_close(out - x32.double().numpy(), ref["out"], "residual step")
+
+
+def test_nonfinite_logit_is_reported():
+    dims = synth.TINY
+    T = 16
+    layer, logits, x, _ = _case(dims, T, seed=55)
+    logits[3, :] = float("nan")
+    _, _, st = run_gpu(layer.to(DEV), x.to(DEV), K=dims.K, logits=logits.to(DEV))
+    assert st == -7
+
+
+def test_bad_precomputed_ids_are_reported_and_contained():
+    dims = synth.TINY
+    T = 12
+    layer = synth.make_layer(dims, seed=56)
+    x = synth.make_x_bf16(T, dims.H, seed=57)
+    ids, w = synth.make_topk(T, dims.E, dims.K, seed=58)
+    ids[2, 0] = 99
+    ids[4, 1] = ids[4, 0]
+    out, _, st = run_gpu(layer.to(DEV), x.to(DEV), K=dims.K, ids=ids.to(DEV), wts=w.to(DEV))
+    assert st == -6
+    assert np.all(out[[2, 4]] == 0.0) and np.all(np.isfinite(out))
+
+
+def test_empty_batch_is_a_noop():
+    import nvfp4_mixture_experts_03_b200 as nv
+    dims = synth.TINY
+    layer = synth.make_layer(dims, seed=59).to(DEV)
+    m = nv.MoELayer.from_layer(layer, top_k=dims.K, max_tokens=16)
+    x = torch.empty(0, dims.H, dtype=torch.bfloat16, device=DEV)
+    out = m.forward(x, logits=torch.empty(0, dims.E, device=DEV))
+    assert out.shape == (0, dims.H) and m.status() == 0
+    m.close()
+
+
+def test_host_checks_on_device():
+    import nvfp4_mixture_experts_03_b200 as nv
+    dims = synth.TINY
+    layer = synth.make_layer(dims, seed=60).to(DEV)
+    m = nv.MoELayer.from_layer(layer, top_k=dims.K, max_tokens=16)
+    x = torch.zeros(17, dims.H, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(nv.NVFP4MoEError) as e:
+        m.forward(x, logits=torch.zeros(17, dims.E, device=DEV))
+    assert e.value.code == -1           # T > max_tokens
+    x = torch.zeros(4, dims.H, dtype=torch.bfloat16, device=DEV)
+    ws = torch.empty(64, dtype=torch.uint8, device=DEV)
+    with pytest.raises(nv.NVFP4MoEError) as e:
+        m.forward(x, logits=torch.zeros(4, dims.E, device=DEV), workspace=ws)
+    assert e.value.code == -4
+    m.close()
