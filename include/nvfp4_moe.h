@@ -197,6 +197,31 @@ NVFP4_MOE_API int nvfp4_moe_get_status(nvfp4_moe_t *h, void *stream);
 #define NVFP4_MOE_PHASE_EVENTS 5
 NVFP4_MOE_API int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events, int32_t n_events);
 
+/* Allocation-free decode call (the pages have no counterpart: this is a service
+ * for callers that cannot allocate device memory at all, and so cannot create a
+ * handle -- nvfp4_moe_create allocates a status block -- or pass a workspace).
+ * It runs the same decode path as nvfp4_moe_forward for 1 <= T <= 8 tokens, with
+ * its scratch in a 1 MiB array compiled into the library (a file-scope
+ * __device__ array: every GPU that loads the library holds it until the process
+ * exits). dims and weights are checked exactly as by nvfp4_moe_create; io and
+ * stream are as for nvfp4_moe_forward. Calls no cudaMalloc/cudaFree.
+ *   - T > 8 returns NVFP4_MOE_ERR_UNSUPPORTED_DIMS; a layer whose decode
+ *     scratch for this T exceeds 1 MiB - 256 bytes returns
+ *     NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL (e.g. H = I = 8192 with K = 16). Both
+ *     are checked before anything is enqueued. T = 0 is a no-op.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress); make that first call before any stream
+ *     capture on the device.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents; each call clears what must start at zero. Calls that overlap on
+ *     the GPU (different streams, or other threads) race on it: serialise them.
+ *   - Device-side routing problems (bad precomputed ids, non-finite logits) are
+ *     contained exactly as in nvfp4_moe_forward but cannot be read back: there
+ *     is no handle, hence no nvfp4_moe_get_status for this call. */
+NVFP4_MOE_API int nvfp4_moe_forward_decode_static(const nvfp4_moe_dims *dims,
+                                                  const nvfp4_moe_weights *weights,
+                                                  const nvfp4_moe_io *io, void *stream);
+
 /* Frees the handle and its status block. Never touches the borrowed weights. */
 NVFP4_MOE_API void nvfp4_moe_destroy(nvfp4_moe_t *h);
 

@@ -30,7 +30,8 @@ MAX_TOPK = 16
 # Every function the header declares (checked against include/nvfp4_moe.h by the tests).
 EXPORTS = ("nvfp4_moe_create", "nvfp4_moe_workspace_bytes", "nvfp4_moe_forward",
            "nvfp4_moe_get_status", "nvfp4_moe_destroy", "nvfp4_moe_strerror",
-           "nvfp4_moe_abi_version", "nvfp4_moe_set_phase_events")
+           "nvfp4_moe_abi_version", "nvfp4_moe_set_phase_events",
+           "nvfp4_moe_forward_decode_static")
 PHASE_EVENTS = 5
 
 
@@ -87,6 +88,9 @@ def lib() -> C.CDLL:
         L.nvfp4_moe_abi_version.restype = C.c_int
         L.nvfp4_moe_set_phase_events.restype = C.c_int
         L.nvfp4_moe_set_phase_events.argtypes = [C.c_void_p, C.POINTER(C.c_void_p), C.c_int32]
+        L.nvfp4_moe_forward_decode_static.restype = C.c_int
+        L.nvfp4_moe_forward_decode_static.argtypes = [C.POINTER(Dims), C.POINTER(Weights),
+                                                      C.POINTER(IO), C.c_void_p]
         _lib = L
     return _lib
 
@@ -133,6 +137,13 @@ def nvfp4_moe_set_phase_events(handle: int, events) -> int:
     """events: sequence of PHASE_EVENTS cudaEvent_t handles (ints), or () to turn off."""
     arr = (C.c_void_p * max(1, len(events)))(*[C.c_void_p(int(e)) for e in events])
     return lib().nvfp4_moe_set_phase_events(C.c_void_p(handle), arr, len(events))
+
+
+def nvfp4_moe_forward_decode_static(dims: Dims, weights: Weights, io: IO, stream: int) -> int:
+    """Allocation-free decode (T <= 8): scratch is a 1 MiB array inside the library,
+    shared by every call on the device -- serialise calls. No handle, no workspace."""
+    return lib().nvfp4_moe_forward_decode_static(C.byref(dims), C.byref(weights), C.byref(io),
+                                                 C.c_void_p(stream))
 
 
 # ------------------------------------------------------------ torch glue

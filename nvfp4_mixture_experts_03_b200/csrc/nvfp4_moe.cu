@@ -11,6 +11,7 @@
 
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "common.cuh"
@@ -324,3 +325,104 @@ void nvfp4_moe_destroy(nvfp4_moe_t *h) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode entry point.
+//
+// For callers that cannot allocate device memory at all -- code running where
+// cudaMalloc is forbidden or unavailable (an allocator-less embedding, a process
+// whose device memory is fully pre-reserved by another runtime) -- and so can
+// neither create a handle (create allocates its status block) nor provide a
+// workspace. The decode path's scratch (routing arrays, F16 activations, h)
+// lives instead in this file-scope device array, which every GPU that loads the
+// library holds until the process exits.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(1) << 20;  // 1 MiB per device
+constexpr size_t kStaticStatusBytes = 256;               // status words, then the workspace
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mu;
+uint8_t *g_static_ptr[kMaxDevices];  // device address of g_static_scratch, per device
+
+// The array's name is only a host-side stand-in; its device address is looked up
+// once per device, with that device current.
+int static_scratch(int dev, uint8_t **out) {
+    if (dev < 0 || dev >= kMaxDevices) return NVFP4_MOE_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p)
+            return NVFP4_MOE_ERR_CUDA;
+        g_static_ptr[dev] = static_cast<uint8_t *>(p);
+    }
+    *out = g_static_ptr[dev];
+    return NVFP4_MOE_OK;
+}
+
+// The same dims/weights checks as nvfp4_moe_create, without its allocation.
+int check_layer(const nvfp4_moe_dims *dims, const nvfp4_moe_weights *w) {
+    if (!dims || !w) return NVFP4_MOE_ERR_INVALID_ARG;
+    const nvfp4_moe_dims d = *dims;
+    if (d.hidden <= 0 || d.inter <= 0 || d.n_experts <= 0 || d.top_k <= 0 || d.max_tokens < 0)
+        return NVFP4_MOE_ERR_INVALID_ARG;
+    if (d.hidden % 128 || d.inter % 128 || d.top_k > d.n_experts ||
+        d.top_k > NVFP4_MOE_MAX_TOPK || d.n_experts > 1024)
+        return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
+    const void *planes[] = {w->gate_codes, w->up_codes, w->gate_scales, w->up_scales,
+                            w->down_codes, w->down_scales};
+    const void *globals[] = {w->gate_global, w->up_global, w->down_global};
+    for (const void *p : planes)
+        if (!p) return NVFP4_MOE_ERR_INVALID_ARG;
+    for (const void *p : globals)
+        if (!p) return NVFP4_MOE_ERR_INVALID_ARG;
+    for (const void *p : planes)
+        if (!al16(p)) return NVFP4_MOE_ERR_MISALIGNED;
+    for (const void *p : globals)
+        if (!al4(p)) return NVFP4_MOE_ERR_MISALIGNED;
+    return NVFP4_MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nvfp4_moe_forward_decode_static(const nvfp4_moe_dims *dims, const nvfp4_moe_weights *w,
+                                    const nvfp4_moe_io *io, void *stream) {
+    int rc = check_layer(dims, w);
+    if (rc != NVFP4_MOE_OK) return rc;
+    if (!io) return NVFP4_MOE_ERR_INVALID_ARG;
+    if (io->T < 0 || io->T > dims->max_tokens) return NVFP4_MOE_ERR_INVALID_ARG;
+    if (io->T > NVFP4_MOE_DECODE_MAX_T) return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
+    if (io->T == 0) return NVFP4_MOE_OK;
+    const size_t need = layout(*dims, io->T).total;
+    if (need > kStaticScratchBytes - kStaticStatusBytes) return NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_MOE_ERR_NO_DEVICE;
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        major != 10)
+        return NVFP4_MOE_ERR_NO_DEVICE;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    uint8_t *scratch = nullptr;
+    rc = static_scratch(dev, &scratch);
+    if (rc != NVFP4_MOE_OK) return rc;
+    // A handle on the stack (allocates nothing) pointing at the static array.
+    nvfp4_moe h;
+    h.d = *dims;
+    h.w = *w;
+    h.device = dev;
+    h.num_sms = sms;
+    h.status = reinterpret_cast<int32_t *>(scratch);
+    h.phase_on = false;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // The status words must start at zero (they latch the first device error).
+    if (cudaMemsetAsync(scratch, 0, kStaticStatusBytes, s) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
+    return nvfp4_moe_forward(&h, io, scratch + kStaticStatusBytes,
+                             kStaticScratchBytes - kStaticStatusBytes, stream);
+}
+
+}  // extern "C"
+
