@@ -44,59 +44,56 @@ def peaks():
 
 
 class Clocks:
-    """Samples nvidia-smi every 100 ms while the timed region runs."""
-    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock and the clock-event (throttle) reasons through NVML
+    every 10 ms while the timed region runs (read-only queries)."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, index: int):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.sm, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self.ok = False
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.index)],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[self.index]) if vis else self.index
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.nv = pynvml
+            self.ok = True
+            self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
-        except OSError:
-            self.proc = None
+        except Exception:
+            self.ok = False
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
 
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if self.ok:
+            self.t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 7:
-                continue
-            try:
-                sm.append(float(f[0]))
-                mx = float(f[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.sm:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(self.sm)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.sm), "via": "NVML, 10 ms"}
 
 
 def dist_setup():
@@ -166,6 +163,8 @@ def run_ours(args, ws, rank, local):
     import nvfp4_mixture_experts_03_b200 as nv
     dev = torch.device("cuda", local)
     pk, pk_src = peaks()
+    if args.decode_only:   # profiling aid: the decode measurement alone
+        return {"metric": METRIC, "decode": run_decode(args, dev, pk, pk_src)}
     wl, layer, logits, x, xs = make_prefill(args.workload, dev)
     d = wl.dims
     T = x.shape[0]
@@ -299,6 +298,9 @@ def run_ours(args, ws, rank, local):
 
 
 def run_decode(args, dev, pk, pk_src):
+    """Decode expert streaming, T in {1,2,4,8}: one step = the layer over each of
+    `decode_layers` distinct layers (so the L2 never holds the weights), captured
+    once as a CUDA graph and replayed."""
     import nvfp4_mixture_experts_03_b200 as nv
     wl = synth.CONFIGS["decode"]
     d = wl.dims
@@ -307,6 +309,7 @@ def run_decode(args, dev, pk, pk_src):
     layers = [synth.make_layer(d, synth.workload_seed(wl, l), device=dev) for l in range(nl)]
     models = [nv.MoELayer.from_layer(L, top_k=d.K, max_tokens=8) for L in layers]
     out = {}
+    reps = max(args.steps, 50)
     for T in wl.tokens:
         xs = [synth.make_x_bf16(T, d.H, synth.workload_seed(wl, l) + 17 * T, outliers=True, device=dev)
               for l in range(nl)]
@@ -319,42 +322,55 @@ def run_decode(args, dev, pk, pk_src):
             models[l].forward(xs[l], logits=lg[l], out=outs[l], debug=dbg)
             uniq += int((dbg["counts"] > 0).sum().item())
         ws_bufs = [mm.workspace(T) for mm in models]
-
-        def step():
-            for l in range(nl):
-                models[l].forward(xs[l], logits=lg[l], out=outs[l], workspace=ws_bufs[l])
-
-        for _ in range(args.warmup):
-            step()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nv.PHASE_EVENTS)]
-               for _ in range(nl * args.steps)]
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nv.PHASE_EVENTS)] for _ in range(nl)]
         for es in evs:
             for e in es:
                 e.record()
         torch.cuda.synchronize()
+        stream = torch.cuda.Stream()
+        stream.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                for l in range(nl):
+                    models[l].forward(xs[l], logits=lg[l], out=outs[l], workspace=ws_bufs[l], stream=stream)
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+                for l in range(nl):
+                    models[l].set_phase_events(evs[l])
+                    models[l].forward(xs[l], logits=lg[l], out=outs[l], workspace=ws_bufs[l], stream=stream)
+                    models[l].set_phase_events(())
+        torch.cuda.current_stream().wait_stream(stream)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        kern_ms = 0.0
         a.record()
-        k = 0
-        for _ in range(args.steps):
-            for l in range(nl):
-                models[l].set_phase_events(evs[k])
-                k += 1
-                models[l].forward(xs[l], logits=lg[l], out=outs[l], workspace=ws_bufs[l])
+        for _ in range(reps):
+            g.replay()
         b.record()
         torch.cuda.synchronize()
-        for mm in models:
-            mm.set_phase_events(())
-        ms = a.elapsed_time(b) / args.steps
-        kern_ms = sum(es[2].elapsed_time(es[4]) for es in evs) / args.steps
+        ms = a.elapsed_time(b) / reps
+        # per-kernel view from the last replay's phase events
+        route_ms = sum(es[0].elapsed_time(es[1]) for es in evs)
+        kern_ms = sum(es[2].elapsed_time(es[4]) for es in evs)
+        for l in range(nl):
+            if models[l].status() != 0:
+                raise RuntimeError(f"decode layer {l} status {models[l].status()}")
+        del g
         nbytes = uniq * per_expert
         gbs = nbytes / (ms / 1e3) / 1e9
         kgbs = nbytes / (kern_ms / 1e3) / 1e9
         out[f"T{T}"] = {"layers": nl, "unique_experts": uniq, "bytes": nbytes,
-                        "layer_us": round(ms * 1e3 / nl, 2), "GBps_layer": round(gbs, 1),
-                        "GBps_expert_kernels": round(kgbs, 1),
+                        "layer_us": round(ms * 1e3 / nl, 2),
+                        "route_us_per_layer": round(route_ms * 1e3 / nl, 2),
+                        "expert_kernels_us_per_layer": round(kern_ms * 1e3 / nl, 2),
+                        "GBps_layer": round(gbs, 1), "GBps_expert_kernels": round(kgbs, 1),
                         "frac_layer": round(gbs / pk["hbm_gbs"], 4),
                         "frac_expert_kernels": round(kgbs / pk["hbm_gbs"], 4)}
     out["peak"] = {"hbm_gbs": pk["hbm_gbs"], "source": pk_src}
+    out["timing"] = "CUDA graph of the 8-layer step, replayed; kernel view from phase events"
     for mm in models:
         mm.close()
     return out
@@ -415,7 +431,7 @@ def run_reference(args, ws, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="prefill8k", choices=["prefill8k", "w4a8_32k"])
@@ -423,6 +439,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-tokens", type=int, default=16)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -193,7 +193,9 @@ NVFP4_MOE_API int nvfp4_moe_get_status(nvfp4_moe_t *h, void *stream);
  * SwiGLU done, 4 down + combine done. (Decode calls stage activations inside
  * routing, so events 1 and 2 coincide.) n_events == 0 turns it off. The handle
  * borrows the events; returns INVALID_ARG for any other n_events. This mirrors
- * per-phase accounting of a layer's time; it adds four event records per call. */
+ * per-phase accounting of a layer's time; it adds five event records per call.
+ * The records are external (cudaEventRecordExternal), so a forward captured into
+ * a CUDA graph records them on every replay. */
 #define NVFP4_MOE_PHASE_EVENTS 5
 NVFP4_MOE_API int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events, int32_t n_events);
 

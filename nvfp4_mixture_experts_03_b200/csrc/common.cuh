@@ -21,7 +21,7 @@ constexpr int kBN = 256;               // max tokens per grouped-GEMM tile (MMA 
 constexpr int kBK = 64;                // K elements per pipeline stage (one 128B swizzle row)
 constexpr int kGuRows = 64;            // intermediate rows per gate/up tile (64 gate + 64 up)
 constexpr int kDnRows = 128;           // hidden rows per down tile
-constexpr int kStages = 4;             // smem pipeline depth of the grouped GEMM
+constexpr int kStages = 4;             // max smem pipeline depth of the grouped GEMM
 
 // Device status block layout (int32 words).
 enum : int { kStatusCode = 0, kStatusDetail = 1, kStatusWords = 16 };
@@ -69,7 +69,7 @@ struct Params {
     Tile *tiles_gu, *tiles_dn;
     int32_t *uniq;             // [<=P] decode: unique experts ascending
     int32_t *upos;             // [<=P][8] decode: position of (unique expert, token) or -1
-    __half *xh;                // prefill: [P][H] permuted activations; decode: [T][H]
+    __half *xh;                // prefill: [P][H] F16 activations per pair position; decode: [T][H]
     __half *h;                 // [P][I]
     int32_t *status;           // device status block
     // optional debug copies
@@ -294,7 +294,8 @@ void launch_route_small(const Params &p, cudaStream_t s);
 void launch_prep_prefill(const Params &p, cudaStream_t s);
 void launch_decode_gateup(const Params &p, cudaStream_t s);
 void launch_decode_down(const Params &p, cudaStream_t s);
-// mode 0: gate/up + SwiGLU over map = F16 activations [P][H]; mode 1: down + combine over map = h [P][I]
+// mode 0: gate/up + SwiGLU, map = F16 activations [P][H]; mode 1: down + combine,
+// map = h [P][I]; both 64 x 64 boxes
 void launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &map, int num_sms,
                          cudaStream_t s);
 cudaError_t prefill_init();   // per device: opt the GEMM kernels into their shared memory

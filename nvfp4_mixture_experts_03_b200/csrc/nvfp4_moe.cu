@@ -48,13 +48,14 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2D F16 tensor [rows][cols], box 64 x 64, 128-byte swizzle, zero fill outside.
-bool make_map_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
+// 2D F16 tensor [rows][cols], box 64 columns x box_rows, 128-byte swizzle, zero
+// fill outside.
+bool make_map_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
     cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kBK, 64};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -263,8 +264,17 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     p.max_tiles_dn = L.max_dn;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // External records, so that a forward captured into a CUDA graph records the
+    // phase events on every replay (a plain record inside capture is only an
+    // ordering dependency).
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (h->phase_on && cudaStreamIsCapturing(s, &cap) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
     auto mark = [&](int i) {
-        if (h->phase_on) cudaEventRecord(h->phase[i], s);
+        if (!h->phase_on) return;
+        if (cap == cudaStreamCaptureStatusActive)
+            cudaEventRecordWithFlags(h->phase[i], s, cudaEventRecordExternal);
+        else
+            cudaEventRecord(h->phase[i], s);
     };
     if (T <= NVFP4_MOE_DECODE_MAX_T) {
         mark(0);
@@ -278,7 +288,7 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     } else {
         const int64_t P = (int64_t)T * d.top_k;
         CUtensorMap map_xh, map_h;
-        if (!make_map_f16(&map_xh, p.xh, P, d.hidden) || !make_map_f16(&map_h, p.h, P, d.inter))
+        if (!make_map_f16(&map_xh, p.xh, P, d.hidden, 64) || !make_map_f16(&map_h, p.h, P, d.inter, 64))
             return NVFP4_MOE_ERR_CUDA;
         mark(0);
         launch_route_large(p, s);

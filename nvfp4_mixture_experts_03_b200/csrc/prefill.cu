@@ -36,6 +36,14 @@ constexpr int kAStage = kBM * kBK * 2;         // 16 KB
 constexpr int kBStage = kBN * kBK * 2;         // 32 KB
 constexpr int kBBox = 64;                      // rows per TMA box
 constexpr int kTmemCols = 512;                 // two 256-column accumulators
+constexpr int kStageBytes = 32 * kBM * 4;      // one epilogue staging buffer: 32 columns x 128 rows x FP32
+// gate/up is bound by the latency of the activation loads: deepest ring, one
+// staging buffer (h chunk). down is bound by its reduction epilogue: 3 stages,
+// 4 staging buffers so bulk reductions of 3 chunks can be in flight.
+template <int MODE> struct Cfg {
+    static constexpr int stages = MODE == 0 ? 4 : 3;
+    static constexpr int bufs = MODE == 0 ? 1 : 4;
+};
 constexpr int kPF = 4;                         // dequant loads in flight (k-steps)
 constexpr uint64_t kDrainNs = 200000000ull;    // bounded drain on abort
 
@@ -50,7 +58,10 @@ struct __align__(8) Bars {
     int abort;
 };
 
-constexpr size_t kSmemBytes = 1024 + kStages * (kAStage + kBStage) + sizeof(Bars);
+template <int MODE>
+constexpr size_t smem_bytes() {
+    return 1024 + Cfg<MODE>::stages * (kAStage + kBStage) + Cfg<MODE>::bufs * kStageBytes + sizeof(Bars);
+}
 
 // Iterates (tile, k-step) pairs of this CTA in order.
 struct Cursor {
@@ -65,11 +76,12 @@ struct Cursor {
     }
 };
 
+template <int S>
 struct Ring {
     int stage = 0;
     uint32_t phase = 0;
     __device__ void next() {
-        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        if (++stage == S) { stage = 0; phase ^= 1; }
     }
 };
 
@@ -117,6 +129,22 @@ __device__ inline void store_row(uint8_t *a_stage, int r, const StepData &d) {
     }
 }
 
+// Named barrier over the four epilogue warps (ids 0 is __syncthreads).
+__device__ inline void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ inline void bulk_reduce_add_f32(float *gdst, const void *ssrc, uint32_t bytes) {
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                     gdst),
+                 "r"(smem_u32(ssrc)), "r"(bytes)
+                 : "memory");
+}
+__device__ inline void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ inline void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ inline void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const Params p, const __grid_constant__ CUtensorMap map_b) {
@@ -124,8 +152,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     uint8_t *a_base = smem;
-    uint8_t *b_base = smem + kStages * kAStage;
-    Bars *bars = reinterpret_cast<Bars *>(b_base + kStages * kBStage);
+    constexpr int S = Cfg<MODE>::stages, NB = Cfg<MODE>::bufs;
+    uint8_t *b_base = smem + S * kAStage;
+    uint8_t *epi_stage = b_base + S * kBStage;                       // NB x kStageBytes
+    Bars *bars = reinterpret_cast<Bars *>(epi_stage + NB * kStageBytes);
     volatile int *abort = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -135,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nk = Kdim / kBK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; s++) {
+        for (int s = 0; s < S; s++) {
             mbar_init(&bars->a_full[s], 128);
             mbar_init(&bars->b_full[s], 1);
             mbar_init(&bars->empty[s], 1);
@@ -162,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ dequantise A rows
         const int r = threadIdx.x - 128;
         Cursor ld(nk, ntiles), cs(nk, ntiles);
-        Ring ring;
+        Ring<S> ring;
         StepData q[kPF];
         int ld_tile = -1;
         const uint8_t *lcodes = nullptr, *lscales = nullptr;
@@ -203,15 +233,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 8) {
         // ------------------------------------------------------ TMA for B
+        // 64-row boxes of the pair-ordered B rows (F16 activations or h) into the
+        // ring; the next tile's descriptor is read one tile ahead.
         if (lane == 0) {
             Cursor cs(nk, ntiles);
-            Ring ring;
+            Ring<S> ring;
             uint32_t issued = 0, issued_phase = 0;  // stages with a load in flight, their parity
+            int cur_tile = -1;
+            Tile t{}, t_n{};
+            if (cs.valid()) t_n = tiles[cs.tile()];
             while (cs.valid()) {
-                const Tile t = tiles[cs.tile()];
-                const int nmma = (t.ntok + 15) & ~15;
-                const int nbox = cdiv(nmma, kBBox);
+                if (cs.tile() != cur_tile) {
+                    cur_tile = cs.tile();
+                    t = t_n;
+                    if (cur_tile + (int)gridDim.x < ntiles) t_n = tiles[cur_tile + (int)gridDim.x];
+                }
                 if (!mbar_wait(&bars->empty[ring.stage], ring.phase ^ 1, abort, p.status, 2)) break;
+                const int nbox = cdiv((t.ntok + 15) & ~15, kBBox);
                 uint8_t *bs = b_base + ring.stage * kBStage;
                 mbar_arrive_expect_tx(&bars->b_full[ring.stage], nbox * kBBox * kBK * 2);
                 for (int b = 0; b < nbox; b++)
@@ -223,14 +261,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cs.next();
             }
             // Every stage's last load must have landed before this CTA may exit.
-            for (int s = 0; s < kStages; s++)
+            for (int s = 0; s < S; s++)
                 if (issued & (1u << s))
                     mbar_wait_drain(&bars->b_full[s], (issued_phase >> s) & 1, kDrainNs);
         }
     } else if (warp == 9) {
         // ----------------------------------------------------- MMA issue
         if (lane == 0) {
-            Ring ring;
+            Ring<S> ring;
             uint32_t acc_phase[2] = {0, 0};
             const int ntl = ntiles > (int)blockIdx.x ? cdiv(ntiles - (int)blockIdx.x, (int)gridDim.x) : 0;
             bool ok = true;
@@ -269,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // -------------------------------------------------------- epilogue
         const int ntl = ntiles > (int)blockIdx.x ? cdiv(ntiles - (int)blockIdx.x, (int)gridDim.x) : 0;
         uint32_t acc_phase[2] = {0, 0};
+        int ep_chunk = 0;
         for (int tl = 0; tl < ntl; tl++) {
             const Tile t = tiles[(int)blockIdx.x + tl * (int)gridDim.x];
             const int buf = tl & 1;
@@ -278,12 +317,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tbase = tmem_base + buf * kBN + ((uint32_t)(warp * 32) << 16);
             const int e = t.expert;
             if (MODE == 0) {
+                // SwiGLU; h staged as [32 columns][64 intermediates] F16, then written
+                // with coalesced 16-byte stores (each column is 128 contiguous bytes of h).
                 const float sg = p.gate_global[e], su = p.up_global[e];
-                const int i = t.m0 + 16 * warp + (lane & 15);
+                const int il = 16 * warp + (lane & 15);
                 const bool is_gate = lane < 16;
+                __half *hs = reinterpret_cast<__half *>(epi_stage);
                 for (int c0 = 0; c0 < t.ntok; c0 += 32) {
                     uint32_t v[32];
                     tmem_ld32(tbase + c0, v);
+                    const float xs_l = (c0 + lane < t.ntok) ? p.ps[t.pos0 + c0 + lane] : 0.0f;
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
@@ -293,37 +336,54 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
                         const float gacc = is_gate ? mine_lo : recv;
                         const float uacc = is_gate ? recv : mine_hi;
-                        const int col = c0 + j + (is_gate ? 0 : 16);
-                        if (col < t.ntok) {
-                            const int pos = t.pos0 + col;
-                            const float xs = p.ps[pos];
-                            const float gv = gacc * sg * xs, uv = uacc * su * xs;
-                            p.h[(size_t)pos * p.I + i] = __float2half_rn(silu(gv) * uv);
-                        }
+                        const int cj = j + (is_gate ? 0 : 16);
+                        const float xs = __shfl_sync(0xffffffffu, xs_l, cj);
+                        const float gv = gacc * sg * xs, uv = uacc * su * xs;
+                        hs[cj * kGuRows + il] = __float2half_rn(silu(gv) * uv);
                     }
+                    epi_sync();
+                    const int ncol = min(32, t.ntok - c0);
+                    for (int q = threadIdx.x; q < ncol * 8; q += 128) {
+                        const int col = q >> 3, part = q & 7;
+                        const uint4 val = reinterpret_cast<const uint4 *>(hs + col * kGuRows)[part];
+                        reinterpret_cast<uint4 *>(p.h + (size_t)(t.pos0 + c0 + col) * p.I + t.m0)[part] = val;
+                    }
+                    epi_sync();
                 }
             } else {
+                // y * s_d * w staged as [32 columns][128 hidden rows] FP32; one bulk
+                // reduction-add per token row segment (512 B) into out.
                 const float sd = p.down_global[e];
-                const int hrow = t.m0 + 32 * warp + lane;
+                const int r = 32 * warp + lane;
                 for (int c0 = 0; c0 < t.ntok; c0 += 32) {
+                    float *st = reinterpret_cast<float *>(epi_stage + (ep_chunk % NB) * kStageBytes);
                     uint32_t v[32];
                     tmem_ld32(tbase + c0, v);
+                    const bool in = c0 + lane < t.ntok;
+                    const float w_l = in ? p.pw[t.pos0 + c0 + lane] * sd : 0.0f;
+                    const int tok_l = (warp == 0 && in) ? p.ptok[t.pos0 + c0 + lane] : 0;
                     tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; j++) {
-                        const int col = c0 + j;
-                        if (col < t.ntok) {
-                            const int pos = t.pos0 + col;
-                            const float w = p.pw[pos] * sd;
-                            atomicAdd(p.out + (size_t)p.ptok[pos] * p.H + hrow,
-                                      __uint_as_float(v[j]) * w);
-                        }
+                    for (int j = 0; j < 32; j++)
+                        st[j * kBM + r] = __uint_as_float(v[j]) * __shfl_sync(0xffffffffu, w_l, j);
+                    fence_proxy_async_smem();
+                    epi_sync();
+                    if (warp == 0) {
+                        // lane j reduces column j; each lane waits for its own earlier
+                        // group to finish reading the other staging buffer
+                        if (in) bulk_reduce_add_f32(p.out + (size_t)tok_l * p.H + t.m0, st + lane * kBM,
+                                                    kBM * 4);
+                        bulk_commit();
+                        bulk_wait_read<NB - 1>();   // the buffer used next is free again
                     }
+                    epi_sync();
+                    ep_chunk++;
                 }
             }
             tc_fence_before();
             mbar_arrive(&bars->acc_empty[buf]);
         }
+        if (MODE == 1 && warp == 0) bulk_wait_all();   // reductions land before exit
     }
 
     tc_fence_before();
@@ -336,18 +396,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t prefill_init() {
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<0>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes<0>());
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kSmemBytes);
+                                (int)smem_bytes<1>());
 }
 
 void launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &map, int num_sms,
                          cudaStream_t s) {
     if (mode == 0)
-        grouped_gemm_kernel<0><<<max(1, min(num_sms, p.max_tiles_gu)), kThreads, kSmemBytes, s>>>(p, map);
+        grouped_gemm_kernel<0><<<max(1, min(num_sms, p.max_tiles_gu)), kThreads, smem_bytes<0>(), s>>>(p, map);
     else
-        grouped_gemm_kernel<1><<<max(1, min(num_sms, p.max_tiles_dn)), kThreads, kSmemBytes, s>>>(p, map);
+        grouped_gemm_kernel<1><<<max(1, min(num_sms, p.max_tiles_dn)), kThreads, smem_bytes<1>(), s>>>(p, map);
 }
 
 }  // namespace nvmoe

@@ -14,50 +14,51 @@
 
 namespace nvmoe {
 
-// Orderable selection key: larger logit first, NaN below every number, equal
-// logits -> lower expert id first. Key 0 marks an already chosen expert.
-__device__ inline unsigned long long sel_key(float v, int e) {
-    uint32_t o;
-    if (isnan(v)) {
-        o = 0;
-    } else {
-        uint32_t u = (v == 0.0f) ? 0u : __float_as_uint(v);
-        o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    }
-    return ((unsigned long long)o << 32) | (uint32_t)(~(uint32_t)e);
+// Orderable 32-bit selection key: larger logit -> larger key; NaN -> 1 (below
+// every number); 0 marks an expert already chosen. +0 and -0 share one key.
+__device__ inline uint32_t sel_key(float v) {
+    if (isnan(v)) return 1u;
+    const uint32_t u = (v == 0.0f) ? 0u : __float_as_uint(v);
+    const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return k < 2u ? 2u : k;  // -inf maps to 0x007FFFFF, so this never changes a number's order
 }
 
-// One warp selects the top-K of one token's logits (E <= 32*NPER). Lane j < K
-// receives the j-th id and its renormalised weight.
+// One warp selects the top-K of one token's logits (E <= 32*NPER): K rounds of
+// (per-lane argmax over its NPER keys, warp max of the key, warp min of the
+// expert id among lanes holding it), so equal logits go to the lower id. Lane
+// j < K receives the j-th id and its renormalised weight.
 template <int NPER>
 __device__ inline void warp_topk(const float *__restrict__ row, int E, int K, int lane,
                                  int &my_id, float &my_w, bool &finite) {
-    unsigned long long key[NPER];
+    uint32_t key[NPER];
+    float val[NPER];
+    // all loads first (clamped in-bounds addresses), so they are in flight together
 #pragma unroll
-    for (int i = 0; i < NPER; i++) {
-        const int e = lane + 32 * i;
-        key[i] = (e < E) ? sel_key(__ldg(row + e), e) : 0ull;
-    }
+    for (int i = 0; i < NPER; i++) val[i] = __ldg(row + min(lane + 32 * i, E - 1));
+#pragma unroll
+    for (int i = 0; i < NPER; i++) key[i] = (lane + 32 * i < E) ? sel_key(val[i]) : 0u;
     my_id = 0;
     float my_v = 0.0f;
     for (int j = 0; j < K; j++) {
-        unsigned long long best = 0;
+        uint32_t best = key[0];
+        int bi = 0;
 #pragma unroll
-        for (int i = 0; i < NPER; i++) best = key[i] > best ? key[i] : best;
+        for (int i = 1; i < NPER; i++)
+            if (key[i] > best) { best = key[i]; bi = i; }   // strict: lowest i (lowest id) on ties
+        const uint32_t gmax = __reduce_max_sync(0xffffffffu, best);
+        const uint32_t cand = (best == gmax) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
+        const int e = (int)__reduce_min_sync(0xffffffffu, cand);
+        const int hit = ((e & 31) == lane) ? (e >> 5) : -1;
+        float v = 0.0f;
 #pragma unroll
-        for (int off = 16; off; off >>= 1) {
-            unsigned long long o = __shfl_xor_sync(0xffffffffu, best, off);
-            best = o > best ? o : best;
+        for (int i = 0; i < NPER; i++) {
+            v = (i == hit) ? val[i] : v;
+            key[i] = (i == hit) ? 0u : key[i];
         }
-        const int e = (int)(~(uint32_t)(best & 0xffffffffull));
-        if ((e & 31) == lane) {
-#pragma unroll
-            for (int i = 0; i < NPER; i++)
-                if (i == (e >> 5)) key[i] = 0ull;
-        }
+        v = __shfl_sync(0xffffffffu, v, e & 31);
         if (lane == j) {
             my_id = e;
-            my_v = __ldg(row + e);
+            my_v = v;
         }
     }
     const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
@@ -106,15 +107,20 @@ __device__ inline void route_token(const Params &p, int t, int lane, int &id, fl
 
 // ---------------------------------------------------------------- large T
 
-// Kernel 1: top-k for 64 tokens per CTA, then the chunk's per-expert counts.
+// Kernel 1: top-k for 64 tokens per CTA (32 warps, 2 tokens each), then the
+// chunk's per-expert counts.
 template <int NPER>
-__global__ void __launch_bounds__(256) route_topk_hist_kernel(Params p) {
+constexpr int topk_threads() { return NPER >= 32 ? 512 : 1024; }
+
+template <int NPER>
+__global__ void __launch_bounds__(topk_threads<NPER>()) route_topk_hist_kernel(Params p) {
     extern __shared__ uint32_t mask[];  // [2][E]
     const int c = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < 2 * p.E; i += blockDim.x) mask[i] = 0;
     __syncthreads();
-    for (int i = 0; i < kChunkTokens / 8; i++) {
-        const int tl = warp * (kChunkTokens / 8) + i;
+    const int per_warp = kChunkTokens / (int)(blockDim.x >> 5);
+    for (int i = 0; i < per_warp; i++) {
+        const int tl = warp * per_warp + i;
         const int t = c * kChunkTokens + tl;
         if (t >= p.T) break;
         int id;
@@ -177,19 +183,19 @@ __device__ int block_exscan(int *a, int n, int *warp_tot /* >= 32 */) {
     return total;
 }
 
-// Writes the gate/up and down tile lists of the experts in [e_begin, e_end).
-__device__ void emit_tiles(const Params &p, const int *cnt_s, const int *off_s, const int *gub,
-                           const int *dnb, int e) {
-    const int c = cnt_s[e];
-    if (c == 0) return;
-    const int nn = cdiv(c, kBN), mgu = p.I / kGuRows, mdn = p.H / kDnRows;
-    for (int nt = 0; nt < nn; nt++) {
-        const int pos0 = off_s[e] + nt * kBN, nk = min(kBN, c - nt * kBN);
-        for (int mi = 0; mi < mgu; mi++)
-            p.tiles_gu[gub[e] + nt * mgu + mi] = Tile{e, mi * kGuRows, pos0, nk};
-        for (int mi = 0; mi < mdn; mi++)
-            p.tiles_dn[dnb[e] + nt * mdn + mi] = Tile{e, mi * kDnRows, pos0, nk};
+// Tile slot -> (expert, n-tile, m-tile) by binary search over the per-expert
+// exclusive tile offsets `base` (E entries, non-decreasing) in shared memory.
+__device__ inline void emit_tile(Tile *tiles, const int *base, const int *cnt_s, const int *off_s,
+                                 int E, int mt, int m_rows, int slot) {
+    int lo = 0, hi = E - 1;  // last e with base[e] <= slot
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (base[mid] <= slot) lo = mid; else hi = mid - 1;
     }
+    const int e = lo, r = slot - base[e];
+    const int nt = r / mt, mi = r - nt * mt;
+    const int pos0 = off_s[e] + nt * kBN;
+    tiles[slot] = Tile{e, mi * m_rows, pos0, min(kBN, cnt_s[e] - nt * kBN)};
 }
 
 // Kernel 2 (one CTA of 1024 threads): per-expert scan over chunks, expert
@@ -245,7 +251,10 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(Params p) {
             if (p.dbg_counts) p.dbg_counts[e] = cnt_s[e];
         }
     }
-    for (int e = threadIdx.x; e < p.E; e += blockDim.x) emit_tiles(p, cnt_s, off_s, gub, dnb, e);
+    for (int slot = threadIdx.x; slot < ngu; slot += blockDim.x)
+        emit_tile(p.tiles_gu, gub, cnt_s, off_s, p.E, mgu, kGuRows, slot);
+    for (int slot = threadIdx.x; slot < ndn; slot += blockDim.x)
+        emit_tile(p.tiles_dn, dnb, cnt_s, off_s, p.E, mdn, kDnRows, slot);
 }
 
 // Kernel 3: positions of every pair of a 64-token chunk.
@@ -277,24 +286,71 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(Params p) {
 
 // --------------------------------------------------------- activations prep
 
-__device__ inline float load_act(const Params &p, int t, int k) {
-    if (p.act_type == NVFP4_MOE_ACT_BF16)
-        return __bfloat162float(((const __nv_bfloat16 *)p.act)[(size_t)t * p.H + k]);
-    if (p.act_type == NVFP4_MOE_ACT_INT8) return (float)((const int8_t *)p.act)[(size_t)t * p.H + k];
-    // FP32 residual stream: the layer's input is its BF16 rounding
-    return __bfloat162float(__float2bfloat16_rn(((const float *)p.act)[(size_t)t * p.H + k]));
+
+// Eight consecutive activations (k8-th group of 8) of token t as FP32, with a
+// 16-byte load (BF16, 8-byte for int8, two 16-byte loads for FP32).
+__device__ inline void load_act8(const Params &p, int t, int k8, float (&v)[8]) {
+    const size_t off = (size_t)t * p.H + 8 * k8;
+    if (p.act_type == NVFP4_MOE_ACT_BF16) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)p.act + off));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    } else if (p.act_type == NVFP4_MOE_ACT_INT8) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2 *>((const int8_t *)p.act + off));
+        const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+        for (int i = 0; i < 8; i++) v[i] = (float)(int8_t)(w[i >> 2] >> (8 * (i & 3)));
+    } else {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>((const float *)p.act + off));
+        const float4 b = __ldg(reinterpret_cast<const float4 *>((const float *)p.act + off) + 1);
+        const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 8; i++) v[i] = __bfloat162float(__float2bfloat16_rn(f[i]));
+    }
+}
+
+// 2^sh as an FP32 (|sh| <= 120, so the exponent field stays normal).
+__device__ inline float exp2i(int sh) { return __int_as_float((127 + sh) << 23); }
+
+__device__ inline uint4 pack8_f16(const float (&v)[8], int sh) {
+    const float m = exp2i(sh);  // exact power-of-two scaling
+    __align__(16) __half hv[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) hv[i] = __float2half_rn(v[i] * m);
+    return *reinterpret_cast<const uint4 *>(hv);
 }
 
 // One CTA per token: F16 copy of x_t scaled by 2^k (BF16/FP32 input) or the int8
-// codes as F16 (exact), written to the position of each of the token's K pairs;
-// the per-position scale that undoes it; and out_t cleared unless accumulating.
+// codes as F16 (exact), written to the position of each of the token's K pairs
+// (the gate/up GEMM then loads contiguous 64-row boxes); the scale that undoes
+// it, per token and per pair position; and out_t cleared unless accumulating.
 __global__ void __launch_bounds__(256) prep_prefill_kernel(Params p) {
     const int t = blockIdx.x;
     __shared__ float red[8];
     __shared__ int spos[NVFP4_MOE_MAX_TOPK];
+    constexpr int kMaxPer = 2;                  // 8-element groups per thread held in registers (H <= 4096)
+    const int n8 = p.H / 8;
+    float v[kMaxPer][8];
     float amax = 0.0f;
-    if (p.act_type != NVFP4_MOE_ACT_INT8)
-        for (int k = threadIdx.x; k < p.H; k += blockDim.x) amax = fmaxf(amax, fabsf(load_act(p, t, k)));
+#pragma unroll
+    for (int i = 0; i < kMaxPer; i++) {
+        const int k8 = threadIdx.x + i * blockDim.x;
+        if (k8 < n8) {
+            load_act8(p, t, k8, v[i]);
+#pragma unroll
+            for (int j = 0; j < 8; j++) amax = fmaxf(amax, fabsf(v[i][j]));
+        }
+    }
+    for (int k8 = threadIdx.x + kMaxPer * blockDim.x; k8 < n8; k8 += blockDim.x) {  // H > 4096
+        float w[8];
+        load_act8(p, t, k8, w);
+#pragma unroll
+        for (int j = 0; j < 8; j++) amax = fmaxf(amax, fabsf(w[j]));
+    }
 #pragma unroll
     for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
@@ -303,20 +359,26 @@ __global__ void __launch_bounds__(256) prep_prefill_kernel(Params p) {
     amax = 0.0f;
     for (int w = 0; w < (int)(blockDim.x >> 5); w++) amax = fmaxf(amax, red[w]);
     const int sh = (p.act_type == NVFP4_MOE_ACT_INT8) ? 0 : pow2_shift_for(amax);
-    const float xs = (p.act_type == NVFP4_MOE_ACT_INT8) ? p.act_scale[t] : ldexpf(1.0f, -sh);
+    const float xs = (p.act_type == NVFP4_MOE_ACT_INT8) ? p.act_scale[t] : exp2i(-sh);
     if (threadIdx.x == 0) p.xscale[t] = xs;
     if (threadIdx.x < p.K) p.ps[spos[threadIdx.x]] = xs;
-    // 8 elements per thread step -> one 16-byte store per pair
-    for (int k8 = threadIdx.x; k8 < p.H / 8; k8 += blockDim.x) {
-        __align__(16) __half v[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) v[i] = __float2half_rn(ldexpf(load_act(p, t, k8 * 8 + i), sh));
-        const uint4 pk = *reinterpret_cast<const uint4 *>(v);
-        for (int j = 0; j < p.K; j++)
-            reinterpret_cast<uint4 *>(p.xh + (size_t)spos[j] * p.H)[k8] = pk;
+    for (int i = 0; i < kMaxPer; i++) {
+        const int k8 = threadIdx.x + i * blockDim.x;
+        if (k8 < n8) {
+            const uint4 pk = pack8_f16(v[i], sh);
+            for (int j = 0; j < p.K; j++) reinterpret_cast<uint4 *>(p.xh + (size_t)spos[j] * p.H)[k8] = pk;
+        }
+    }
+    for (int k8 = threadIdx.x + kMaxPer * blockDim.x; k8 < n8; k8 += blockDim.x) {
+        float w[8];
+        load_act8(p, t, k8, w);
+        const uint4 pk = pack8_f16(w, sh);
+        for (int j = 0; j < p.K; j++) reinterpret_cast<uint4 *>(p.xh + (size_t)spos[j] * p.H)[k8] = pk;
     }
     if (!p.out_add)
-        for (int k = threadIdx.x; k < p.H; k += blockDim.x) p.out[(size_t)t * p.H + k] = 0.0f;
+        for (int k4 = threadIdx.x; k4 < p.H / 4; k4 += blockDim.x)
+            reinterpret_cast<float4 *>(p.out + (size_t)t * p.H)[k4] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // ---------------------------------------------------------------- small T
@@ -324,8 +386,10 @@ __global__ void __launch_bounds__(256) prep_prefill_kernel(Params p) {
 // One CTA, T <= 8: routing, counts, offsets, permutation, the unique-expert list
 // with each (unique expert, token) position, the F16 activations and the
 // output clear, in one launch.
+constexpr int kSmallThreads = 512;
+
 template <int NPER>
-__global__ void __launch_bounds__(256) route_small_kernel(Params p) {
+__global__ void __launch_bounds__(kSmallThreads) route_small_kernel(Params p) {
     extern __shared__ int sm[];
     int *emask = sm;                  // [E] token bitmask per expert
     int *cnt_s = emask + p.E;         // [E] counts -> offsets
@@ -333,9 +397,10 @@ __global__ void __launch_bounds__(256) route_small_kernel(Params p) {
     int *wt = flag + p.E;             // [33]
     __shared__ int sid[NVFP4_MOE_DECODE_MAX_T * NVFP4_MOE_MAX_TOPK];
     __shared__ float sw[NVFP4_MOE_DECODE_MAX_T * NVFP4_MOE_MAX_TOPK];
-    __shared__ float samax[NVFP4_MOE_DECODE_MAX_T];
+    __shared__ unsigned samax_u[NVFP4_MOE_DECODE_MAX_T];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) emask[e] = 0;
+    if (threadIdx.x < NVFP4_MOE_DECODE_MAX_T) samax_u[threadIdx.x] = 0u;
     __syncthreads();
     if (warp < p.T) {
         const int t = warp;
@@ -351,24 +416,35 @@ __global__ void __launch_bounds__(256) route_small_kernel(Params p) {
             if (p.dbg_w) p.dbg_w[t * p.K + lane] = w;
             atomicOr(&emask[id], 1 << t);
         }
-        // activation amax of this token (for the F16 shift)
-        float amax = 0.0f;
-        if (p.act_type != NVFP4_MOE_ACT_INT8)
-            for (int k = lane; k < p.H; k += 32) amax = fmaxf(amax, fabsf(load_act(p, t, k)));
+    }
+    // per-token activation amax (for the F16 shift): 16-byte loads from all threads
+    if (p.act_type != NVFP4_MOE_ACT_INT8) {
+        const int n8 = p.H / 8;
+#pragma unroll 4
+        for (int c = threadIdx.x; c < p.T * n8; c += blockDim.x) {
+            float v[8];
+            load_act8(p, c / n8, c % n8, v);
+            float m = 0.0f;
 #pragma unroll
-        for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        if (lane == 0) samax[t] = amax;
+            for (int j = 0; j < 8; j++) m = fmaxf(m, fabsf(v[j]));
+            atomicMax(&samax_u[c / n8], __float_as_uint(m));   // non-negative: integer order
+        }
     }
     __syncthreads();
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
-        cnt_s[e] = __popc(emask[e]);
-        flag[e] = emask[e] != 0;
-        p.counts[e] = cnt_s[e];
-        if (p.dbg_counts) p.dbg_counts[e] = cnt_s[e];
+        const int c = __popc(emask[e]);
+        cnt_s[e] = c | ((c != 0) << 16);   // one scan: pairs (low 16 bits), used experts (high)
+        p.counts[e] = c;
+        if (p.dbg_counts) p.dbg_counts[e] = c;
     }
     __syncthreads();
-    const int total = block_exscan(cnt_s, p.E, wt);
-    const int U = block_exscan(flag, p.E, wt);
+    const int both = block_exscan(cnt_s, p.E, wt);
+    const int total = both & 0xFFFF, U = both >> 16;
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+        flag[e] = cnt_s[e] >> 16;
+        cnt_s[e] &= 0xFFFF;
+    }
+    __syncthreads();
     if (threadIdx.x == 0) {
         p.cnt[kCntUniq] = U;
         p.offsets[p.E] = total;
@@ -396,14 +472,24 @@ __global__ void __launch_bounds__(256) route_small_kernel(Params p) {
         p.pw[pos] = sw[q];
         if (p.dbg_perm) p.dbg_perm[pos] = q;
     }
-    for (int t = 0; t < p.T; t++) {
-        const int sh = (p.act_type == NVFP4_MOE_ACT_INT8) ? 0 : pow2_shift_for(samax[t]);
-        if (threadIdx.x == 0)
-            p.xscale[t] = (p.act_type == NVFP4_MOE_ACT_INT8) ? p.act_scale[t] : ldexpf(1.0f, -sh);
-        for (int k = threadIdx.x; k < p.H; k += blockDim.x)
-            p.xh[(size_t)t * p.H + k] = __float2half_rn(ldexpf(load_act(p, t, k), sh));
+    if (threadIdx.x < p.T) {
+        const int t = threadIdx.x;
+        const int sh = (p.act_type == NVFP4_MOE_ACT_INT8) ? 0 : pow2_shift_for(__uint_as_float(samax_u[t]));
+        p.xscale[t] = (p.act_type == NVFP4_MOE_ACT_INT8) ? p.act_scale[t] : exp2i(-sh);
+    }
+    {
+        const int n8 = p.H / 8;
+#pragma unroll 4
+        for (int c = threadIdx.x; c < p.T * n8; c += blockDim.x) {
+            const int t = c / n8;
+            const int sh = (p.act_type == NVFP4_MOE_ACT_INT8) ? 0 : pow2_shift_for(__uint_as_float(samax_u[t]));
+            float v[8];
+            load_act8(p, t, c % n8, v);
+            reinterpret_cast<uint4 *>(p.xh)[c] = pack8_f16(v, sh);
+        }
         if (!p.out_add)
-            for (int k = threadIdx.x; k < p.H; k += blockDim.x) p.out[(size_t)t * p.H + k] = 0.0f;
+            for (int c = threadIdx.x; c < p.T * p.H / 4; c += blockDim.x)
+                reinterpret_cast<float4 *>(p.out)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 
@@ -422,7 +508,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(Params p) {
 
 void launch_route_large(const Params &p, cudaStream_t s) {
     const size_t mask_bytes = 2 * p.E * sizeof(uint32_t);
-    NPER_SWITCH(p.E, (route_topk_hist_kernel<NP><<<p.nch, 256, mask_bytes, s>>>(p)));
+    NPER_SWITCH(p.E, (route_topk_hist_kernel<NP><<<p.nch, topk_threads<NP>(), mask_bytes, s>>>(p)));
     const size_t scan_bytes = (4 * p.E + 1 + 33) * sizeof(int);
     route_scan_kernel<<<1, 1024, scan_bytes, s>>>(p);
     route_scatter_kernel<<<p.nch, 256, mask_bytes, s>>>(p);
@@ -434,7 +520,7 @@ void launch_prep_prefill(const Params &p, cudaStream_t s) {
 
 void launch_route_small(const Params &p, cudaStream_t s) {
     const size_t bytes = (3 * p.E + 33) * sizeof(int);
-    NPER_SWITCH(p.E, (route_small_kernel<NP><<<1, 256, bytes, s>>>(p)));
+    NPER_SWITCH(p.E, (route_small_kernel<NP><<<1, kSmallThreads, bytes, s>>>(p)));
 }
 
 }  // namespace nvmoe
