@@ -290,7 +290,6 @@ __device__ inline int pow2_shift_for(float amax) {
 
 // ------------------------------------------------------------ kernel decls
 void launch_route_large(const Params &p, cudaStream_t s);
-void launch_route_small(const Params &p, cudaStream_t s);
 void launch_prep_prefill(const Params &p, cudaStream_t s);
 void launch_decode_gateup(const Params &p, cudaStream_t s);
 void launch_decode_down(const Params &p, cudaStream_t s);
@@ -299,5 +298,6 @@ void launch_decode_down(const Params &p, cudaStream_t s);
 void launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &map, int num_sms,
                          cudaStream_t s);
 cudaError_t prefill_init();   // per device: opt the GEMM kernels into their shared memory
+cudaError_t decode_init();    // per device: opt the decode kernels into their shared memory
 
 }  // namespace nvmoe

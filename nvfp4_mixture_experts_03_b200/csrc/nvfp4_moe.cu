@@ -105,7 +105,7 @@ WsLayout layout(const nvfp4_moe_dims &d, int T) {
     L.tiles_dn = take((size_t)L.max_dn * sizeof(Tile));
     L.uniq = take(decode ? P * 4 : 0);
     L.upos = take(decode ? P * NVFP4_MOE_DECODE_MAX_T * 4 : 0);
-    L.xh = take((decode ? (size_t)T : P) * d.hidden * 2);
+    L.xh = take(decode ? 0 : P * d.hidden * 2);   // decode stages activations in shared memory
     L.h = take(P * d.inter * 2);
     L.total = o;
     return L;
@@ -162,7 +162,8 @@ int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (major != 10) return NVFP4_MOE_ERR_NO_DEVICE;
-    if (prefill_init() != cudaSuccess || !encode_fn()) return NVFP4_MOE_ERR_CUDA;
+    if (prefill_init() != cudaSuccess || decode_init() != cudaSuccess || !encode_fn())
+        return NVFP4_MOE_ERR_CUDA;
     nvfp4_moe *h = new (std::nothrow) nvfp4_moe;
     if (!h) return NVFP4_MOE_ERR_CUDA;
     h->d = d;
@@ -277,8 +278,9 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
             cudaEventRecord(h->phase[i], s);
     };
     if (T <= NVFP4_MOE_DECODE_MAX_T) {
+        // routing happens inside both decode kernels (every CTA routes the <= 8
+        // tokens itself), so phases 0-2 coincide
         mark(0);
-        launch_route_small(p, s);
         mark(1);
         mark(2);
         launch_decode_gateup(p, s);
