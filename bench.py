@@ -242,7 +242,16 @@ def run_ours(args, ws, rank, local):
                       "l2": "inputs larger than L2 (1.27 GiB of expert planes per layer)",
                       "parallelism": f"replicas x{ws}"},
            "roofline": roof, "phases": phases, "clocks": clk.summary(),
-           "gpu_launches": 6 * args.steps}
+           "gpu_launches": 7 * args.steps}
+
+    if wl.act == "int8":
+        # the same tokens through the BF16-activation path (informational)
+        xf = synth.make_x_f32(T, d.H, synth.workload_seed(wl), outliers=wl.outliers, device=dev)
+        ob = m.forward(xf.to(torch.bfloat16), logits=logits)
+        oi = m.forward(x, logits=logits, x_scale=xs)
+        res["w4a8_vs_bf16_rel_l2"] = round(float(torch.linalg.vector_norm((oi - ob).double()) /
+                                                 torch.linalg.vector_norm(ob.double())), 5)
+        del xf, ob, oi
 
     # ---- end to end: host buffers, copies inside the timed region
     if not args.no_e2e:
@@ -275,7 +284,7 @@ def run_ours(args, ws, rank, local):
         h2d = xh.numel() * xh.element_size() + lh.numel() * 4 + (xsh.numel() * 4 if xsh is not None else 0)
         res["e2e"] = {"value": round(ws * T * args.steps / (e_ms / 1e3), 1), "unit": "tok/s",
                       "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(oh.numel() * 4)}
-        res["gpu_launches"] += 6 * args.steps
+        res["gpu_launches"] += 7 * args.steps
 
     # ---- decode expert GB/s (8 distinct layers so the L2 never holds the weights)
     if not args.no_decode:
@@ -378,12 +387,109 @@ def profile_traffic(kernel_key):
     return rec["dram_bytes_per_launch"] if h == rec["source_sha256_16"] else None
 
 
+def run_stack(args, ws, rank, local):
+    """48 stacked layers (independent seeds), x <- x + layer(bf16(x)) carried in
+    FP32 in place. Prefill: one step = the 4096-token chunk through all 48 layers.
+    Decode: T = 1..4 through all 48 layers, captured as one CUDA graph."""
+    import nvfp4_mixture_experts_03_b200 as nv
+    dev = torch.device("cuda", local)
+    pk, pk_src = peaks()
+    wl = synth.CONFIGS["stack48"]
+    d = wl.dims
+    t0 = time.perf_counter()
+    layers = [synth.make_layer(d, synth.workload_seed(wl, l), device=dev) for l in range(wl.layers)]
+    gen_s = time.perf_counter() - t0
+    Tp = 4096
+    models = [nv.MoELayer.from_layer(L, top_k=d.K, max_tokens=Tp) for L in layers]
+    wsb = models[0].workspace(Tp)                  # one workspace shared by the sequential layers
+    lgp = [synth.make_logits(Tp, d.E, synth.workload_seed(wl, l) + 202, zipf_s=wl.zipf_s, device=dev)
+           for l in range(wl.layers)]
+    x0 = synth.make_x_f32(Tp, d.H, synth.workload_seed(wl) + 2, outliers=False, device=dev).contiguous()
+    x = x0.clone()
+
+    def step():
+        x.copy_(x0)
+        for l in range(wl.layers):
+            models[l].forward(x, logits=lgp[l], out=x, accumulate=True, workspace=wsb)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(1, args.steps // 20)
+    with Clocks(dev.index) as clk:
+        a.record()
+        for _ in range(steps):
+            step()
+        b.record()
+        torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), ws) / steps
+    for mm in models:
+        assert mm.status() == 0
+    flops = 2.0 * Tp * d.K * 3 * d.I * d.H * wl.layers
+    res = {"metric": METRIC, "value": round(ws * Tp / (ms / 1e3), 1), "unit": "tok/s",
+           "n_gpus": ws, "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f16 (exact NVFP4 dequant, FP32 accumulate)", "data": "synthetic",
+           "config": {"workload": f"stack48: {wl.note}; prefill chunk {Tp} tokens",
+                      "resident_expert_bytes": sum(L.nbytes() for L in layers),
+                      "generation_s": round(gen_s, 1),
+                      "l2": "inputs larger than L2 (61 GiB of expert planes)"},
+           "stack_tflops": round(flops / (ms / 1e3) / 1e12, 1), "clocks": clk.summary(),
+           "gpu_launches": 7 * wl.layers * steps}
+    # decode through the whole stack, T = 1..4, one CUDA graph per T
+    per_expert = (3 * d.I * d.H) // 2 + (3 * d.I * d.H) // 16
+    dec = {}
+    for T in (1, 2, 3, 4):
+        xd0 = synth.make_x_f32(T, d.H, synth.workload_seed(wl) + 1 + T, outliers=False, device=dev).contiguous()
+        xd = xd0.clone()
+        lgd = [synth.make_logits(T, d.E, synth.workload_seed(wl, l) + 101 + T, zipf_s=wl.zipf_s,
+                                 device=dev) for l in range(wl.layers)]
+        uniq = 0
+        for l in range(wl.layers):
+            dbg = nv.debug_buffers(T, d.E, d.K, dev)
+            models[l].forward(xd, logits=lgd[l], out=xd, accumulate=True, workspace=wsb, debug=dbg)
+            uniq += int((dbg["counts"] > 0).sum().item())
+        st = torch.cuda.Stream()
+        st.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(st):
+            with torch.cuda.graph(g, stream=st, capture_error_mode="thread_local"):
+                xd.copy_(xd0)
+                for l in range(wl.layers):
+                    models[l].forward(xd, logits=lgd[l], out=xd, accumulate=True, workspace=wsb, stream=st)
+        torch.cuda.current_stream().wait_stream(st)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        reps = 20
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        dms = a.elapsed_time(b) / reps
+        gbs = uniq * per_expert / (dms / 1e3) / 1e9
+        dec[f"T{T}"] = {"tokens_per_s": round(T / (dms / 1e3), 1), "ms_per_token_step": round(dms, 3),
+                        "unique_experts": uniq, "GBps": round(gbs, 1), "frac": round(gbs / pk["hbm_gbs"], 4)}
+        del g
+    dec["peak"] = {"hbm_gbs": pk["hbm_gbs"], "source": pk_src}
+    res["decode_stack"] = dec
+    for mm in models:
+        mm.close()
+    return res
+
+
 # --------------------------------------------------------- reference (oracle) arm
 
 def run_reference(args, ws, rank):
     if rank != 0:
         return None
-    wl = synth.CONFIGS[args.workload]
+    # the 48-layer stack's layers have the 8K layer's shape: the oracle's cost per
+    # token and layer is the same, so its stack rate is the layer rate / 48
+    per_layers = 48 if args.workload == "stack48" else 1
+    wl = synth.CONFIGS["prefill8k" if args.workload == "stack48" else args.workload]
     d = wl.dims
     seed = synth.workload_seed(wl)
     T = wl.tokens[0]
@@ -402,7 +508,7 @@ def run_reference(args, ws, rank):
     for _ in range(args.steps):
         cpu_oracle_rate(layer, x, logits, d.K, n, xs)
     dt = time.perf_counter() - t0
-    v = n * args.steps / dt
+    v = n * args.steps / dt / per_layers
     return {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tok/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt * 1e3 / args.steps, 2), "higher_is_better": True,
@@ -410,7 +516,8 @@ def run_reference(args, ws, rank):
             "config": {"workload": f"{wl.name}: {wl.note}", "tokens_per_step": n},
             "cpu_baseline": {"value": round(v, 3), "unit": "tok/s", "cores": os.cpu_count(),
                              "kind": "oracle",
-                             "sample": f"first {n} tokens of the {T}-token chunk per step"},
+                             "sample": f"first {n} tokens of the {T}-token chunk per step"
+                                       + (", one layer; rate divided by 48 layers" if per_layers > 1 else "")},
             "e2e": {"value": round(v, 3), "unit": "tok/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -421,7 +528,7 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="prefill8k", choices=["prefill8k", "w4a8_32k"])
+    ap.add_argument("--workload", default="prefill8k", choices=["prefill8k", "w4a8_32k", "stack48"])
     ap.add_argument("--decode-layers", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-tokens", type=int, default=16)
@@ -434,6 +541,8 @@ def main():
     ws, rank, local = dist_setup()
     if args.impl == "reference":
         res = run_reference(args, ws, rank)
+    elif args.workload == "stack48":
+        res = run_stack(args, ws, rank, local)
     else:
         res = run_ours(args, ws, rank, local)
     if rank == 0 and res is not None:

@@ -73,14 +73,17 @@ extern "C" {
 #define NVFP4_MOE_API
 #endif
 
-/* Largest top-k the kernels support, and the largest T the decode path takes. */
+/* Largest top-k the kernels support, the largest T the decode path takes, and
+ * the largest max_tokens a handle accepts. */
 #define NVFP4_MOE_MAX_TOPK 16
 #define NVFP4_MOE_DECODE_MAX_T 8
+#define NVFP4_MOE_MAX_TOKENS 65536
 
 typedef enum {
     NVFP4_MOE_OK = 0,
     NVFP4_MOE_ERR_INVALID_ARG = -1,        /* null pointer, T<0, T>max_tokens, bad enum   */
-    NVFP4_MOE_ERR_UNSUPPORTED_DIMS = -2,   /* H or I not a multiple of 128; K>E; K>16; E>1024 */
+    NVFP4_MOE_ERR_UNSUPPORTED_DIMS = -2,   /* H or I not a multiple of 128; K>E; K>16; E>1024;
+                                              max_tokens > 65536                              */
     NVFP4_MOE_ERR_MISALIGNED = -3,         /* a plane or buffer not 16-byte aligned       */
     NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL = -4,
     NVFP4_MOE_ERR_CUDA = -5,               /* a CUDA runtime/driver call failed           */

@@ -144,7 +144,7 @@ int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
     if (d.hidden % 128 || d.inter % 128 || d.top_k > d.n_experts ||
         d.top_k > NVFP4_MOE_MAX_TOPK || d.n_experts > 1024)
         return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
-    if ((int64_t)d.max_tokens * d.top_k > (1 << 30)) return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
+    if (d.max_tokens > NVFP4_MOE_MAX_TOKENS) return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
     const void *planes[] = {w->gate_codes, w->up_codes, w->gate_scales, w->up_scales,
                             w->down_codes, w->down_scales};
     const void *globals[] = {w->gate_global, w->up_global, w->down_global};
@@ -381,7 +381,7 @@ int check_layer(const nvfp4_moe_dims *dims, const nvfp4_moe_weights *w) {
     if (d.hidden <= 0 || d.inter <= 0 || d.n_experts <= 0 || d.top_k <= 0 || d.max_tokens < 0)
         return NVFP4_MOE_ERR_INVALID_ARG;
     if (d.hidden % 128 || d.inter % 128 || d.top_k > d.n_experts ||
-        d.top_k > NVFP4_MOE_MAX_TOPK || d.n_experts > 1024)
+        d.top_k > NVFP4_MOE_MAX_TOPK || d.n_experts > 1024 || d.max_tokens > NVFP4_MOE_MAX_TOKENS)
         return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
     const void *planes[] = {w->gate_codes, w->up_codes, w->gate_scales, w->up_scales,
                             w->down_codes, w->down_scales};

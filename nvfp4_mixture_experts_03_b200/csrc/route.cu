@@ -64,8 +64,39 @@ __device__ inline void emit_tile(Tile *tiles, const int *base, const int *cnt_s,
     tiles[slot] = Tile{e, mi * m_rows, pos0, min(kBN, cnt_s[e] - nt * kBN)};
 }
 
-// Kernel 2 (one CTA of 1024 threads): per-expert scan over chunks, expert
-// offsets, and the grouped-GEMM tile lists.
+// Kernel 2: one warp per expert: exclusive scan of its per-chunk counts (all
+// loads issued first) -> cbase[e][c], and the expert's total -> counts[e].
+__global__ void __launch_bounds__(1024) route_chunkscan_kernel(Params p) {
+    const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (e >= p.E) return;
+    const int *__restrict__ hrow = p.hist + (size_t)e * p.nch;
+    int *__restrict__ crow = p.cbase + (size_t)e * p.nch;
+    constexpr int kMaxIt = 32;   // nch <= 1024 chunks (T <= 65536)
+    int v[kMaxIt];
+#pragma unroll
+    for (int i = 0; i < kMaxIt; i++) {
+        const int c = 32 * i + lane;
+        v[i] = c < p.nch ? hrow[c] : 0;
+    }
+    int carry = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxIt; i++) {
+        if (32 * i >= p.nch) break;
+        int incl = v[i];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
+        }
+        const int c = 32 * i + lane;
+        if (c < p.nch) crow[c] = carry + incl - v[i];
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) p.counts[e] = carry;
+}
+
+// Kernel 3 (one CTA of 1024 threads): expert offsets and the grouped-GEMM tile
+// lists.
 __global__ void __launch_bounds__(1024) route_scan_kernel(Params p) {
     extern __shared__ int sm[];
     int *cnt_s = sm;                      // [E]
@@ -73,25 +104,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(Params p) {
     int *gub = off_s + p.E + 1;           // [E]
     int *dnb = gub + p.E;                 // [E]
     int *wt = dnb + p.E;                  // [33]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    for (int e = warp; e < p.E; e += nw) {
-        int carry = 0;
-        const int *hrow = p.hist + (size_t)e * p.nch;
-        int *crow = p.cbase + (size_t)e * p.nch;
-        for (int c0 = 0; c0 < p.nch; c0 += 32) {
-            const int c = c0 + lane;
-            const int v = c < p.nch ? hrow[c] : 0;
-            int incl = v;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                int o = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += o;
-            }
-            if (c < p.nch) crow[c] = carry + incl - v;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) cnt_s[e] = carry;
-    }
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) cnt_s[e] = p.counts[e];
     __syncthreads();
     const int mgu = p.I / kGuRows, mdn = p.H / kDnRows;
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
@@ -112,10 +125,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(Params p) {
     for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
         p.offsets[e] = off_s[e];
         if (p.dbg_offsets) p.dbg_offsets[e] = off_s[e];
-        if (e < p.E) {
-            p.counts[e] = cnt_s[e];
-            if (p.dbg_counts) p.dbg_counts[e] = cnt_s[e];
-        }
+        if (e < p.E && p.dbg_counts) p.dbg_counts[e] = cnt_s[e];
     }
     for (int slot = threadIdx.x; slot < ngu; slot += blockDim.x)
         emit_tile(p.tiles_gu, gub, cnt_s, off_s, p.E, mgu, kGuRows, slot);
@@ -123,7 +133,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(Params p) {
         emit_tile(p.tiles_dn, dnb, cnt_s, off_s, p.E, mdn, kDnRows, slot);
 }
 
-// Kernel 3: positions of every pair of a 64-token chunk.
+// Kernel 4: positions of every pair of a 64-token chunk.
 __global__ void __launch_bounds__(256) route_scatter_kernel(Params p) {
     extern __shared__ uint32_t mask[];  // [2][E]
     const int c = blockIdx.x;
@@ -226,6 +236,7 @@ __global__ void __launch_bounds__(256) prep_prefill_kernel(Params p) {
 void launch_route_large(const Params &p, cudaStream_t s) {
     const size_t mask_bytes = 2 * p.E * sizeof(uint32_t);
     NPER_SWITCH(p.E, (route_topk_hist_kernel<NP><<<p.nch, topk_threads<NP>(), mask_bytes, s>>>(p)));
+    route_chunkscan_kernel<<<cdiv(p.E, 32), 1024, 0, s>>>(p);
     const size_t scan_bytes = (4 * p.E + 1 + 33) * sizeof(int);
     route_scan_kernel<<<1, 1024, scan_bytes, s>>>(p);
     route_scatter_kernel<<<p.nch, 256, mask_bytes, s>>>(p);

@@ -103,6 +103,14 @@ def bf16_rne(v: float) -> int:
     return lib().orc_bf16_rne(C.c_double(v))
 
 
+def bf16_rne_array(v) -> np.ndarray:
+    """FP64 array -> BF16 bits (uint16), each the nearest BF16, ties to even."""
+    a = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+    out = np.zeros(a.shape, np.uint16)
+    lib().orc_bf16_rne_array(C.c_int64(a.size), _p(a), _p(out))
+    return out
+
+
 def route(logits, K: int):
     """-> (ids int32 [T][K], w float64 [T][K], n_nonfinite_tokens)"""
     l = _np(logits).astype(np.float32, copy=False)

@@ -83,6 +83,10 @@ uint16_t orc_bf16_rne(double v) {
     return best;
 }
 
+void orc_bf16_rne_array(int64_t n, const double *v, uint16_t *out) {
+    for (int64_t i = 0; i < n; i++) out[i] = orc_bf16_rne(v[i]);
+}
+
 /* Tables built from the decoders above, once. */
 static double g_e2m1[16], g_e4m3[256];
 static pthread_once_t g_once = PTHREAD_ONCE_INIT;

@@ -45,6 +45,7 @@ double orc_e2m1(uint32_t nibble);
 double orc_e4m3(uint32_t byte);       /* NaN for 0x7F / 0xFF */
 double orc_bf16(uint16_t bits);
 uint16_t orc_bf16_rne(double v);      /* nearest BF16, ties to even */
+void orc_bf16_rne_array(int64_t n, const double *v, uint16_t *out);
 
 /* Top-K of FP32 logits (NaN ranks below everything, ties -> lower id), ordered
  * descending; w[t][j] = exp(l_j - l_max) / sum over the K selected. Returns the

@@ -57,6 +57,7 @@ def _weights(align=256):
     ((2048, 768, 2048, 10, 64), -2),             # E > 1024
     ((2048, 768, 512, 0, 64), -1),               # K = 0
     ((2048, 768, 512, 10, -1), -1),              # negative max_tokens
+    ((2048, 768, 512, 10, 65537), -2),           # max_tokens above the routing scan's limit
 ])
 def test_create_validates_dims_before_device(L, dims, code):
     h = C.c_void_p(123)

@@ -74,6 +74,17 @@ def test_bf16_rne_vs_torch():
         assert oracle.bf16_rne(v) == r, (v, oracle.bf16_rne(v), r)
 
 
+def test_bf16_rne_array_matches_scalar():
+    g = np.random.default_rng(7)
+    v = g.standard_normal(5000) * np.exp2(g.integers(-30, 30, 5000))
+    bits = oracle.bf16_rne_array(v)
+    assert all(int(b) == oracle.bf16_rne(float(x)) for b, x in zip(bits[:500], v[:500]))
+    # a value exactly halfway between two BF16 neighbours, in FP64 only (no FP32 detour)
+    lo = 1.0 + 2.0 ** -7                # BF16 1.0078125 (odd last bit)
+    assert oracle.bf16_rne_array(np.array([lo + 2.0 ** -8]))[0] == 0x3F82   # tie -> even (1.015625)
+    assert oracle.bf16_rne_array(np.array([1.0 + 2.0 ** -8 + 2.0 ** -40]))[0] == 0x3F81
+
+
 def test_dequant_products_exact_in_fp16_and_bf16():
     """code x scale has at most 6 significant bits and lies in [2^-10, 2688]: it is
     exact in both 16-bit float formats (checked exhaustively over 16 x 126 pairs)."""
