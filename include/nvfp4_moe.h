@@ -43,7 +43,7 @@
  *   - Every pointer in nvfp4_moe_weights and nvfp4_moe_io is a DEVICE pointer
  *     owned by the caller. The handle BORROWS the weight pointers: they must stay
  *     valid until nvfp4_moe_destroy. The library allocates no device memory
- *     except one 64-byte status block made by nvfp4_moe_create.
+ *     except one 256-byte status block made by nvfp4_moe_create.
  *   - All scratch lives in the caller's workspace (nvfp4_moe_workspace_bytes).
  *
  * Errors: every call returns 0 (NVFP4_MOE_OK) or a negative nvfp4_moe_status.

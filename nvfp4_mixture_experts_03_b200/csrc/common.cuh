@@ -23,8 +23,11 @@ constexpr int kGuRows = 64;            // intermediate rows per gate/up tile (64
 constexpr int kDnRows = 128;           // hidden rows per down tile
 constexpr int kStages = 4;             // max smem pipeline depth of the grouped GEMM
 
-// Device status block layout (int32 words).
-enum : int { kStatusCode = 0, kStatusDetail = 1, kStatusWords = 16 };
+// Device status block layout (int32 words, 256 bytes): the latched error and its
+// detail, and the decode kernel's grid-wide barrier (generation word, top-level
+// arrival count, kBarGroups group arrival counts).
+enum : int { kStatusCode = 0, kStatusDetail = 1, kStatusBarGen = 8, kStatusBarTop = 9,
+             kStatusBarGroup = 16, kBarGroups = 16, kStatusWords = 64 };
 
 // Per-call routing/tile counters kept in the workspace (int32 words).
 enum : int { kCntTilesGu = 0, kCntTilesDn = 1, kCntUniq = 2, kCntWords = 64 };
@@ -291,8 +294,7 @@ __device__ inline int pow2_shift_for(float amax) {
 // ------------------------------------------------------------ kernel decls
 void launch_route_large(const Params &p, cudaStream_t s);
 void launch_prep_prefill(const Params &p, cudaStream_t s);
-void launch_decode_gateup(const Params &p, cudaStream_t s);
-void launch_decode_down(const Params &p, cudaStream_t s);
+cudaError_t launch_decode(const Params &p, cudaStream_t s);   // the whole T <= 8 layer
 // mode 0: gate/up + SwiGLU, map = F16 activations [P][H]; mode 1: down + combine,
 // map = h [P][I]; both 64 x 64 boxes
 void launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &map, int num_sms,

@@ -130,22 +130,15 @@ __device__ void cta_route(const Params &p, DecRoute &R, int *emask, int *cnt, bo
         R.total = both & 0xFFFF;
         R.U = both >> 16;
     }
-    for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
-        const int m = emask[e];
-        if (!m) continue;
-        const int u = cnt[e] >> 16, off = cnt[e] & 0xFFFF;
-        R.uniq[u] = e;
-        for (int t = 0; t < kSlots; t++) {
-            int pos = -1;
-            float wt = 0.0f;
-            if ((m >> t) & 1) {
-                pos = off + __popc(m & ((1 << t) - 1));
-                for (int j = 0; j < p.K; j++)
-                    if (R.ids[t * p.K + j] == e) wt = R.w[t * p.K + j];
-            }
-            R.upos[u * kSlots + t] = pos;
-            R.uw[u * kSlots + t] = wt;
-        }
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
+        if (emask[e]) R.uniq[cnt[e] >> 16] = e;
+    for (int i = threadIdx.x; i < kMaxUniq * kSlots; i += blockDim.x) R.upos[i] = -1;
+    __syncthreads();
+    for (int q = threadIdx.x; q < p.T * p.K; q += blockDim.x) {   // one thread per (token, slot)
+        const int t = q / p.K, e = R.ids[q];
+        const int u = cnt[e] >> 16;
+        R.upos[u * kSlots + t] = (cnt[e] & 0xFFFF) + __popc(emask[e] & ((1 << t) - 1));
+        R.uw[u * kSlots + t] = R.w[q];
     }
     __syncthreads();
 }
@@ -233,36 +226,89 @@ __device__ inline void issue_loads(const Params &p, const ItemRef &it, int g, in
     }
 }
 
-// MODE 0: gate/up + SwiGLU. Item = (unique expert u, 8 intermediate rows): A
-//   rows g are gate rows, rows g+8 the up rows of the same intermediate index, so
-//   each thread ends with g and u of the same (row, token) pair.
-// MODE 1: down + weighted combine. Item = (unique expert u, 16 hidden rows); the
-//   B operand is h of the pairs (token, u), zero for tokens not routed to u.
-// Persistent CTAs: each pass covers kDecWarps/split items; the weight loads of
-// the next pass are issued before the current pass computes (two register
-// buffers), so every warp keeps its HBM stream going across passes.
-template <int MODE, int NPER>
-__global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(Params p) {
-    extern __shared__ __align__(16) uint8_t dsm[];
-    __shared__ DecRoute R;
-    // gate/up may start before the previous grid (for instance the one that wrote
-    // the router logits) has finished: it waits before reading any input, and
-    // only then lets its dependent (the down kernel) launch. The down kernel's
-    // predecessor is this gate/up grid, which writes none of the routing inputs
-    // or weights, so it routes and starts its weight stream before waiting.
-    if (MODE == 0) grid_dep_wait();
-    grid_dep_launch();
+// Grid-wide barrier for a cooperatively launched grid (all CTAs co-resident),
+// used once per kernel. Each CTA reads the generation word, then arrives on the
+// count; the last to arrive advances the generation (which the others poll) and
+// only then resets the count, so the release costs two dependent atomics and the
+// words (in the handle's device status block) are ready for the next launch. The
+// wait is bounded: after `limit_ns` it latches NVFP4_MOE_ERR_TIMEOUT and returns.
+__device__ inline void grid_barrier_once(int32_t *status, uint64_t limit_ns = 200000000ull) {
+    unsigned *gen = reinterpret_cast<unsigned *>(status + kStatusBarGen);
+    unsigned *count = reinterpret_cast<unsigned *>(status + kStatusBarTop);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        volatile unsigned *vgen = gen;
+        const unsigned my_gen = *vgen;
+        __threadfence();
+        if (atomicAdd(count, 1u) + 1u == gridDim.x) {
+            atomicAdd(gen, 1u);
+            atomicExch(count, 0u);
+        } else {
+            const uint64_t t0 = globaltimer();
+            while (*vgen == my_gen) {
+                __nanosleep(20);
+                if (globaltimer() - t0 > limit_ns) {
+                    latch_status(status, NVFP4_MOE_ERR_TIMEOUT, 100);
+                    break;
+                }
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+}
+
+struct DecSmem {
+    float *red;     // [8 warps][32][4] split-K partial sums
+    __half *xs;     // [8 token slots][H+4] F16 activations
+    uint8_t *raw;   // [T][H] raw BF16 / int8 activations (cp.async at kernel start)
+};
+
+__device__ inline void cp_async16(void *smem, const void *gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+                 : "memory");
+}
+
+// Raw activation bytes per token held in shared memory (0: FP32 input, which is
+// read from global memory instead).
+__host__ __device__ inline int raw_act_bytes(int act_type, int H) {
+    return act_type == NVFP4_MOE_ACT_BF16 ? 2 * H : (act_type == NVFP4_MOE_ACT_INT8 ? H : 0);
+}
+
+// Eight activations of token t (group k8) as FP32, from the shared raw copy when
+// there is one, else from global memory.
+__device__ inline void act8(const Params &p, const uint8_t *raw, int t, int k8, float (&v)[8]) {
+    if (p.act_type == NVFP4_MOE_ACT_BF16) {
+        const uint4 u = reinterpret_cast<const uint4 *>(raw + (size_t)t * 2 * p.H)[k8];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    } else if (p.act_type == NVFP4_MOE_ACT_INT8) {
+        const uint2 u = reinterpret_cast<const uint2 *>(raw + (size_t)t * p.H)[k8];
+        const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+        for (int i = 0; i < 8; i++) v[i] = (float)(int8_t)(w[i >> 2] >> (8 * (i & 3)));
+    } else {
+        load_act8(p, t, k8, v);
+    }
+}
+
+// The weight-streaming passes of one projection over this CTA's share of the
+// items. MODE 0: gate/up + SwiGLU; item = (unique expert u, 8 intermediate rows):
+// A rows g are gate rows, rows g+8 the up rows of the same intermediate index,
+// so each thread ends with g and u of the same (row, token) pair. MODE 1: down +
+// weighted combine; item = (unique expert u, 16 hidden rows); B = h of the pairs
+// (token, u), zero for tokens not routed to u. Each pass covers kDecWarps/split
+// items; the next pass's loads are issued before the current pass computes (two
+// register buffers). On entry buf0 already holds this CTA's first pass.
+template <int MODE>
+__device__ inline void run_passes(const Params &p, const DecRoute &R, const DecSmem &S,
+                                  PassBuf &buf0, PassBuf &buf1) {
     const int H = p.H, I = p.I, T = p.T;
-    float *red = reinterpret_cast<float *>(dsm);                               // [8][32][4]
-    int *emask = reinterpret_cast<int *>(dsm + kDecWarps * 32 * 4 * sizeof(float));
-    int *cnt = emask + p.E;
-    __half *xs = reinterpret_cast<__half *>(cnt + p.E);                        // [8][H+4] (MODE 0)
-    const int ld = H + 4;
-
-    cta_route<NPER>(p, R, emask, cnt, blockIdx.x == 0);
-
-    const int Kd = MODE == 0 ? H : I;
-    const int rounds = Kd / 128;
+    const int rounds = (MODE == 0 ? H : I) / 128;
     const int split = k_split(rounds);
     const int rpw = cdiv(rounds, split);
     const int ipc = kDecWarps / split;
@@ -271,57 +317,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(Params p) {
     const int item_l = warp / split, part = warp % split;
     const int r_begin = part * rpw, r_end = min(rounds, r_begin + rpw);
     const int stride = gridDim.x * ipc;
-
-    PassBuf buf0, buf1;
+    const int ld = H + 4;
+    const __half *xrow = S.xs + g * ld + 32 * q;
     int base = blockIdx.x * ipc;
     ItemRef cur = item_ref<MODE>(p, R, base + item_l, items);
-    issue_loads<MODE>(p, cur, g, q, r_begin, r_end, buf0);
 
-    // down: from here on it reads h, written by the gate/up grid
-    if (MODE == 1) grid_dep_wait();
-    if (MODE == 0) {
-        // per-token amax -> power-of-two shift -> F16 activations of the 8 token
-        // slots (zeros past T) in shared memory
-        if (threadIdx.x < kSlots) R.amax[threadIdx.x] = 0u;
-        __syncthreads();
-        const int n8 = H / 8;
-        if (p.act_type != NVFP4_MOE_ACT_INT8) {
-            for (int c = threadIdx.x; c < T * n8; c += blockDim.x) {
-                float v[8];
-                load_act8(p, c / n8, c % n8, v);
-                float m = 0.0f;
-#pragma unroll
-                for (int j = 0; j < 8; j++) m = fmaxf(m, fabsf(v[j]));
-                atomicMax(&R.amax[c / n8], __float_as_uint(m));
-            }
-        }
-        __syncthreads();
-        for (int c = threadIdx.x; c < kSlots * n8; c += blockDim.x) {
-            const int t = c / n8, k8 = c % n8;
-            uint4 pk = make_uint4(0, 0, 0, 0);
-            if (t < T) {
-                const int sh = p.act_type == NVFP4_MOE_ACT_INT8 ? 0 : pow2_shift_for(__uint_as_float(R.amax[t]));
-                float v[8];
-                load_act8(p, t, k8, v);
-                pk = pack8_f16(v, sh);
-            }
-            uint2 *d = reinterpret_cast<uint2 *>(xs + t * ld + 8 * k8);
-            d[0] = make_uint2(pk.x, pk.y);
-            d[1] = make_uint2(pk.z, pk.w);
-        }
-        if (threadIdx.x < T)
-            R.xsc[threadIdx.x] = p.act_type == NVFP4_MOE_ACT_INT8
-                                     ? p.act_scale[threadIdx.x]
-                                     : exp2i(-pow2_shift_for(__uint_as_float(R.amax[threadIdx.x])));
-        if (blockIdx.x == 0) publish_route(p, R, emask, cnt);
-        if (!p.out_add)   // clear out for the down kernel's reductions, split over the grid
-            for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < T * H / 4; c += gridDim.x * blockDim.x)
-                reinterpret_cast<float4 *>(p.out)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-        __syncthreads();
-    }
-    const __half *xrow = xs + g * ld + 32 * q;
-
-    // one pass: compute from b while the next pass's loads fill nb
     auto pass_step = [&](PassBuf &b, PassBuf &nb) {
         const ItemRef nxt = item_ref<MODE>(p, R, base + stride + item_l, items);
         issue_loads<MODE>(p, nxt, g, q, r_begin, r_end, nb);
@@ -358,12 +358,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(Params p) {
             }
         }
         if (split > 1) {
-            *reinterpret_cast<float4 *>(red + (warp * 32 + lane) * 4) =
+            *reinterpret_cast<float4 *>(S.red + (warp * 32 + lane) * 4) =
                 make_float4(acc[0], acc[1], acc[2], acc[3]);
             __syncthreads();
             if (part == 0) {
                 for (int w2 = 1; w2 < split; w2++) {
-                    const float4 o = *reinterpret_cast<const float4 *>(red + ((warp + w2) * 32 + lane) * 4);
+                    const float4 o = *reinterpret_cast<const float4 *>(S.red + ((warp + w2) * 32 + lane) * 4);
                     acc[0] += o.x;
                     acc[1] += o.y;
                     acc[2] += o.z;
@@ -407,6 +407,113 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(Params p) {
     }
 }
 
+template <int MODE>
+__device__ inline void first_loads(const Params &p, const DecRoute &R, PassBuf &b) {
+    const int rounds = (MODE == 0 ? p.H : p.I) / 128;
+    const int split = k_split(rounds);
+    const int rpw = cdiv(rounds, split);
+    const int ipc = kDecWarps / split;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int items = R.U * ((MODE == 0 ? p.I : p.H) / (MODE == 0 ? 8 : 16));
+    const int part = warp % split, r_begin = part * rpw;
+    const ItemRef it = item_ref<MODE>(p, R, blockIdx.x * ipc + warp / split, items);
+    issue_loads<MODE>(p, it, lane >> 2, lane & 3, r_begin, min(rounds, r_begin + rpw), b);
+}
+
+// The whole decode layer in one cooperatively launched grid: every CTA routes
+// the <= 8 tokens itself, stages the F16 activations, streams its share of the
+// gate/up weights (SwiGLU into h), issues its first down-projection loads, and
+// after one grid-wide barrier (h complete, out cleared) streams its share of the
+// down weights with the weighted combine.
+template <int NPER>
+__global__ void __launch_bounds__(kDecThreads, 2) decode_layer_kernel(Params p) {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ DecRoute R;
+    const int H = p.H, T = p.T;
+    DecSmem S;
+    S.red = reinterpret_cast<float *>(dsm);
+    int *emask = reinterpret_cast<int *>(dsm + kDecWarps * 32 * 4 * sizeof(float));
+    int *cnt = emask + p.E;
+    S.xs = reinterpret_cast<__half *>(cnt + p.E);
+    S.raw = reinterpret_cast<uint8_t *>(S.xs + kSlots * (H + 4));
+    const int ld = H + 4;
+
+    // the activations first: their loads are then not queued behind the weights'
+    const int raw_bytes = T * raw_act_bytes(p.act_type, H);
+    for (int c = threadIdx.x; c < raw_bytes / 16; c += blockDim.x)
+        cp_async16(S.raw + 16 * c, static_cast<const uint8_t *>(p.act) + 16 * c);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+
+    cta_route<NPER>(p, R, emask, cnt, blockIdx.x == 0);
+    PassBuf buf0, buf1;
+    first_loads<0>(p, R, buf0);
+
+    // per-token amax -> power-of-two shift -> F16 activations in shared memory
+    // (token slots past T are zeros); every load of x is issued before its use
+    const int n8 = H / 8;
+    for (int c = threadIdx.x; c < (kSlots - T) * n8; c += blockDim.x) {
+        uint2 *dst = reinterpret_cast<uint2 *>(S.xs + (T + c / n8) * ld + 8 * (c % n8));
+        dst[0] = make_uint2(0, 0);
+        dst[1] = make_uint2(0, 0);
+    }
+    if (threadIdx.x < kSlots) R.amax[threadIdx.x] = 0u;
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    // two passes over the shared raw copy (global memory for FP32 input): the
+    // per-token amax (reduced per warp, one shared atomic per warp and token),
+    // then the shifted F16 values. Loop bounds are whole warps for the shuffles.
+    const int ngrp = T * n8, ngrp_w = (ngrp + 31) & ~31;
+    if (p.act_type != NVFP4_MOE_ACT_INT8) {
+        for (int c = threadIdx.x; c < ngrp_w; c += blockDim.x) {
+            float m = 0.0f;
+            if (c < ngrp) {
+                float v[8];
+                act8(p, S.raw, c / n8, c % n8, v);
+#pragma unroll
+                for (int j = 0; j < 8; j++) m = fmaxf(m, fabsf(v[j]));
+            }
+            // a warp's 32 groups span at most two tokens (n8 is a multiple of 16)
+            const unsigned t = (unsigned)min(c / n8, kSlots - 1);
+            const unsigned lo_t = __shfl_sync(0xffffffffu, t, 0);
+            const unsigned hi_t = __reduce_max_sync(0xffffffffu, t);
+            const unsigned mb = __float_as_uint(m);
+            const unsigned m_lo = __reduce_max_sync(0xffffffffu, t == lo_t ? mb : 0u);
+            const unsigned m_hi = __reduce_max_sync(0xffffffffu, t != lo_t ? mb : 0u);
+            if ((threadIdx.x & 31) == 0) {
+                if (lo_t < (unsigned)T) atomicMax(&R.amax[lo_t], m_lo);
+                if (hi_t != lo_t && hi_t < (unsigned)T) atomicMax(&R.amax[hi_t], m_hi);
+            }
+        }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < ngrp; c += blockDim.x) {
+        const int t = c / n8;
+        const int sh = p.act_type == NVFP4_MOE_ACT_INT8 ? 0 : pow2_shift_for(__uint_as_float(R.amax[t]));
+        float v[8];
+        act8(p, S.raw, t, c % n8, v);
+        const uint4 pk = pack8_f16(v, sh);
+        uint2 *dst = reinterpret_cast<uint2 *>(S.xs + t * ld + 8 * (c % n8));
+        dst[0] = make_uint2(pk.x, pk.y);
+        dst[1] = make_uint2(pk.z, pk.w);
+    }
+    if (threadIdx.x < T)
+        R.xsc[threadIdx.x] = p.act_type == NVFP4_MOE_ACT_INT8
+                                 ? p.act_scale[threadIdx.x]
+                                 : exp2i(-pow2_shift_for(__uint_as_float(R.amax[threadIdx.x])));
+    if (blockIdx.x == 0) publish_route(p, R, emask, cnt);
+    // out is cleared for the combine before the grid barrier below; act never
+    // aliases out in this mode (only an accumulating call may pass act == out)
+    if (!p.out_add)
+        for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < T * H / 4; c += gridDim.x * blockDim.x)
+            reinterpret_cast<float4 *>(p.out)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
+
+    run_passes<0>(p, R, S, buf0, buf1);
+    first_loads<1>(p, R, buf0);     // down weights in flight while the grid catches up
+    grid_barrier_once(p.status);    // h complete, out cleared
+    run_passes<1>(p, R, S, buf0, buf1);
+}
+
 static int sm_count() {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -414,49 +521,49 @@ static int sm_count() {
     return sms;
 }
 
-template <int MODE, int NPER>
-static void launch_one(const Params &p, cudaStream_t s) {
-    const int U_max = min(p.T * p.K, p.E);
-    const int rounds = (MODE == 0 ? p.H : p.I) / 128;
-    const int ipc = kDecWarps / k_split(rounds);
-    const int items = U_max * (MODE == 0 ? p.I / 8 : p.H / 16);
-    const size_t smem = kDecWarps * 32 * 4 * sizeof(float) + 2 * (size_t)p.E * sizeof(int) +
-                        (MODE == 0 ? (size_t)8 * (p.H + 4) * sizeof(__half) : 0);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(max(1, min(2 * sm_count(), cdiv(items, ipc))));
-    cfg.blockDim = dim3(kDecThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, decode_kernel<MODE, NPER>, p);
+static size_t decode_smem(const Params &p) {
+    return kDecWarps * 32 * 4 * sizeof(float) + 2 * (size_t)p.E * sizeof(int) +
+           (size_t)8 * (p.H + 4) * sizeof(__half) + (size_t)p.T * raw_act_bytes(p.act_type, p.H);
 }
 
-#define DEC_NPER_SWITCH(E, MODE)                                                  \
-    do {                                                                          \
-        const int _n = cdiv((E), 32);                                             \
-        if (_n <= 1) launch_one<MODE, 1>(p, s);                                   \
-        else if (_n <= 2) launch_one<MODE, 2>(p, s);                              \
-        else if (_n <= 4) launch_one<MODE, 4>(p, s);                              \
-        else if (_n <= 8) launch_one<MODE, 8>(p, s);                              \
-        else if (_n <= 16) launch_one<MODE, 16>(p, s);                            \
-        else launch_one<MODE, 32>(p, s);                                          \
-    } while (0)
+template <int NPER>
+static cudaError_t launch_layer(const Params &p, cudaStream_t s) {
+    const size_t smem = decode_smem(p);
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_layer_kernel<NPER>,
+                                                                  kDecThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int U_max = min(p.T * p.K, p.E);
+    const int need = max(cdiv(U_max * (p.I / 8), kDecWarps / k_split(p.H / 128)),
+                         cdiv(U_max * (p.H / 16), kDecWarps / k_split(p.I / 128)));
+    const int grid = max(1, min(min(per_sm, 2) * sm_count(), need));
+    Params pp = p;
+    void *args[] = {&pp};
+    return cudaLaunchCooperativeKernel((const void *)decode_layer_kernel<NPER>, dim3(grid),
+                                       dim3(kDecThreads), args, smem, s);
+}
 
-void launch_decode_gateup(const Params &p, cudaStream_t s) { DEC_NPER_SWITCH(p.E, 0); }
-void launch_decode_down(const Params &p, cudaStream_t s) { DEC_NPER_SWITCH(p.E, 1); }
+cudaError_t launch_decode(const Params &p, cudaStream_t s) {
+    const int n = cdiv(p.E, 32);
+    if (n <= 1) return launch_layer<1>(p, s);
+    if (n <= 2) return launch_layer<2>(p, s);
+    if (n <= 4) return launch_layer<4>(p, s);
+    if (n <= 8) return launch_layer<8>(p, s);
+    if (n <= 16) return launch_layer<16>(p, s);
+    return launch_layer<32>(p, s);
+}
 
 cudaError_t decode_init() {
-    // dynamic shared memory above 48 KB for the gate/up kernel at large H
+    // dynamic shared memory above 48 KB (the F16 activations grow with H)
     const int big = 200 * 1024;
-#define DEC_ATTR(M, N) cudaFuncSetAttribute(decode_kernel<M, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, big)
-    const cudaError_t r[] = {DEC_ATTR(0, 1), DEC_ATTR(0, 2), DEC_ATTR(0, 4), DEC_ATTR(0, 8),
-                             DEC_ATTR(0, 16), DEC_ATTR(0, 32), DEC_ATTR(1, 1), DEC_ATTR(1, 2),
-                             DEC_ATTR(1, 4), DEC_ATTR(1, 8), DEC_ATTR(1, 16), DEC_ATTR(1, 32)};
-#undef DEC_ATTR
+    const cudaError_t r[] = {
+        cudaFuncSetAttribute(decode_layer_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
+        cudaFuncSetAttribute(decode_layer_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
+        cudaFuncSetAttribute(decode_layer_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
+        cudaFuncSetAttribute(decode_layer_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
+        cudaFuncSetAttribute(decode_layer_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
+        cudaFuncSetAttribute(decode_layer_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big)};
     for (cudaError_t x : r)
         if (x != cudaSuccess) return x;
     return cudaSuccess;

@@ -278,14 +278,13 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
             cudaEventRecord(h->phase[i], s);
     };
     if (T <= NVFP4_MOE_DECODE_MAX_T) {
-        // routing happens inside both decode kernels (every CTA routes the <= 8
-        // tokens itself), so phases 0-2 coincide
+        // one kernel for the whole decode layer: its routing, staging and both
+        // projections are not separable by events (phases 0-2 and 3-4 coincide)
         mark(0);
         mark(1);
         mark(2);
-        launch_decode_gateup(p, s);
+        if (launch_decode(p, s) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
         mark(3);
-        launch_decode_down(p, s);
         mark(4);
     } else {
         const int64_t P = (int64_t)T * d.top_k;
