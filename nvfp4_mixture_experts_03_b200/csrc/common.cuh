@@ -72,7 +72,8 @@ struct Params {
     Tile *tiles_gu, *tiles_dn;
     int32_t *uniq;             // [<=P] decode: unique experts ascending
     int32_t *upos;             // [<=P][8] decode: position of (unique expert, token) or -1
-    __half *xh;                // prefill: [P][H] F16 activations per pair position; decode: [T][H]
+    __half *xh;                // prefill: [P][H] F16 activations per pair position, then the
+                               // down projection's w * s_d * y per pair (F16)
     __half *h;                 // [P][I]
     int32_t *status;           // device status block
     // optional debug copies
@@ -294,6 +295,7 @@ __device__ inline int pow2_shift_for(float amax) {
 // ------------------------------------------------------------ kernel decls
 void launch_route_large(const Params &p, cudaStream_t s);
 void launch_prep_prefill(const Params &p, cudaStream_t s);
+void launch_combine(const Params &p, cudaStream_t s);   // prefill: per-token sum of the K pair rows
 cudaError_t launch_decode(const Params &p, cudaStream_t s);   // the whole T <= 8 layer
 // mode 0: gate/up + SwiGLU, map = F16 activations [P][H]; mode 1: down + combine,
 // map = h [P][I]; both 64 x 64 boxes

@@ -299,6 +299,7 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
         launch_prefill_gemm(0, p, map_xh, h->num_sms, s);
         mark(3);
         launch_prefill_gemm(1, p, map_h, h->num_sms, s);
+        launch_combine(p, s);
         mark(4);
     }
     return cudaGetLastError() == cudaSuccess ? NVFP4_MOE_OK : NVFP4_MOE_ERR_CUDA;

@@ -20,7 +20,8 @@
 // Epilogues: gate/up -> scales, SwiGLU, F16 h at the pair's position (64 gate
 // rows and 64 up rows of the same intermediate indices share a tile, arranged
 // so that each TMEM lane quarter holds 16 gate and the matching 16 up rows);
-// down -> scale x routing weight, FP32 reduction-add into out[token].
+// down -> scale x routing weight, F16 row per pair (combined per token by a
+// separate deterministic kernel).
 //
 // Warp roles (320 threads): 0-3 epilogue, 4-7 dequantise A, 8 TMA for B,
 // 9 TMEM allocation + MMA issue. Every mbarrier wait is bounded (2 s); on
@@ -37,12 +38,11 @@ constexpr int kBStage = kBN * kBK * 2;         // 32 KB
 constexpr int kBBox = 64;                      // rows per TMA box
 constexpr int kTmemCols = 512;                 // two 256-column accumulators
 constexpr int kStageBytes = 32 * kBM * 4;      // one epilogue staging buffer: 32 columns x 128 rows x FP32
-// gate/up is bound by the latency of the activation loads: deepest ring, one
-// staging buffer (h chunk). down is bound by its reduction epilogue: 3 stages,
-// 4 staging buffers so bulk reductions of 3 chunks can be in flight.
+// Both GEMMs: a 4-stage ring and one epilogue staging buffer (a 32-column chunk
+// of h, or of the down projection's per-pair F16 rows).
 template <int MODE> struct Cfg {
-    static constexpr int stages = MODE == 0 ? 4 : 3;
-    static constexpr int bufs = MODE == 0 ? 1 : 4;
+    static constexpr int stages = 4;
+    static constexpr int bufs = 1;
 };
 constexpr int kPF = 4;                         // dequant loads in flight (k-steps)
 constexpr uint64_t kDrainNs = 200000000ull;    // bounded drain on abort
@@ -131,19 +131,6 @@ __device__ inline void store_row(uint8_t *a_stage, int r, const StepData &d) {
 
 // Named barrier over the four epilogue warps (ids 0 is __syncthreads).
 __device__ inline void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-__device__ inline void bulk_reduce_add_f32(float *gdst, const void *ssrc, uint32_t bytes) {
-    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                     gdst),
-                 "r"(smem_u32(ssrc)), "r"(bytes)
-                 : "memory");
-}
-__device__ inline void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-template <int N>
-__device__ inline void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-__device__ inline void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -307,7 +294,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // -------------------------------------------------------- epilogue
         const int ntl = ntiles > (int)blockIdx.x ? cdiv(ntiles - (int)blockIdx.x, (int)gridDim.x) : 0;
         uint32_t acc_phase[2] = {0, 0};
-        int ep_chunk = 0;
         for (int tl = 0; tl < ntl; tl++) {
             const Tile t = tiles[(int)blockIdx.x + tl * (int)gridDim.x];
             const int buf = tl & 1;
@@ -351,39 +337,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     epi_sync();
                 }
             } else {
-                // y * s_d * w staged as [32 columns][128 hidden rows] FP32; one bulk
-                // reduction-add per token row segment (512 B) into out.
+                // y * s_d * w staged as [32 columns][128 hidden rows] F16, written with
+                // coalesced 16-byte stores into the pair's row of yp; the combine
+                // kernel sums each token's K rows in a fixed order.
                 const float sd = p.down_global[e];
                 const int r = 32 * warp + lane;
+                __half *ys = reinterpret_cast<__half *>(epi_stage);
                 for (int c0 = 0; c0 < t.ntok; c0 += 32) {
-                    float *st = reinterpret_cast<float *>(epi_stage + (ep_chunk % NB) * kStageBytes);
                     uint32_t v[32];
                     tmem_ld32(tbase + c0, v);
-                    const bool in = c0 + lane < t.ntok;
-                    const float w_l = in ? p.pw[t.pos0 + c0 + lane] * sd : 0.0f;
-                    const int tok_l = (warp == 0 && in) ? p.ptok[t.pos0 + c0 + lane] : 0;
+                    const float w_l = (c0 + lane < t.ntok) ? p.pw[t.pos0 + c0 + lane] * sd : 0.0f;
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 32; j++)
-                        st[j * kBM + r] = __uint_as_float(v[j]) * __shfl_sync(0xffffffffu, w_l, j);
-                    fence_proxy_async_smem();
+                        ys[j * kBM + r] = __float2half_rn(__uint_as_float(v[j]) * __shfl_sync(0xffffffffu, w_l, j));
                     epi_sync();
-                    if (warp == 0) {
-                        // lane j reduces column j; each lane waits for its own earlier
-                        // group to finish reading the other staging buffer
-                        if (in) bulk_reduce_add_f32(p.out + (size_t)tok_l * p.H + t.m0, st + lane * kBM,
-                                                    kBM * 4);
-                        bulk_commit();
-                        bulk_wait_read<NB - 1>();   // the buffer used next is free again
+                    const int ncol = min(32, t.ntok - c0);
+                    for (int q = threadIdx.x; q < ncol * (kBM / 8); q += 128) {
+                        const int col = q / (kBM / 8), part = q % (kBM / 8);
+                        const uint4 val = reinterpret_cast<const uint4 *>(ys + col * kBM)[part];
+                        reinterpret_cast<uint4 *>(p.xh + (size_t)(t.pos0 + c0 + col) * p.H + t.m0)[part] = val;
                     }
                     epi_sync();
-                    ep_chunk++;
                 }
             }
             tc_fence_before();
             mbar_arrive(&bars->acc_empty[buf]);
         }
-        if (MODE == 1 && warp == 0) bulk_wait_all();   // reductions land before exit
     }
 
     tc_fence_before();

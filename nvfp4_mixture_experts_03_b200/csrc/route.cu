@@ -165,8 +165,8 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(Params p) {
 
 // One CTA per token: F16 copy of x_t scaled by 2^k (BF16/FP32 input) or the int8
 // codes as F16 (exact), written to the position of each of the token's K pairs
-// (the gate/up GEMM then loads contiguous 64-row boxes); the scale that undoes
-// it, per token and per pair position; and out_t cleared unless accumulating.
+// (the gate/up GEMM then loads contiguous 64-row boxes); and the scale that
+// undoes it, per token and per pair position.
 __global__ void __launch_bounds__(256) prep_prefill_kernel(Params p) {
     const int t = blockIdx.x;
     __shared__ float red[8];
@@ -215,9 +215,52 @@ __global__ void __launch_bounds__(256) prep_prefill_kernel(Params p) {
         const uint4 pk = pack8_f16(w, sh);
         for (int j = 0; j < p.K; j++) reinterpret_cast<uint4 *>(p.xh + (size_t)spos[j] * p.H)[k8] = pk;
     }
-    if (!p.out_add)
-        for (int k4 = threadIdx.x; k4 < p.H / 4; k4 += blockDim.x)
-            reinterpret_cast<float4 *>(p.out + (size_t)t * p.H)[k4] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// -------------------------------------------------------------- combine
+
+// out_t (+)= sum_j yp[pos(t, j)] over the token's K pairs, in the fixed order
+// j = 0..K-1 with FP32 accumulation (yp holds w * s_d * y per pair, F16, in the
+// buffer that held the pair-ordered activations). One CTA per token; each thread
+// issues all K loads of its 8 columns before adding them up.
+__global__ void __launch_bounds__(256) combine_kernel(Params p) {
+    const int t = blockIdx.x;
+    __shared__ int spos[NVFP4_MOE_MAX_TOPK];
+    if (threadIdx.x < p.K) spos[threadIdx.x] = p.inv[(size_t)t * p.K + threadIdx.x];
+    __syncthreads();
+    for (int k8 = threadIdx.x; k8 < p.H / 8; k8 += blockDim.x) {
+        uint4 y[NVFP4_MOE_MAX_TOPK];
+#pragma unroll
+        for (int j = 0; j < NVFP4_MOE_MAX_TOPK; j++)
+            if (j < p.K) y[j] = reinterpret_cast<const uint4 *>(p.xh + (size_t)spos[j] * p.H)[k8];
+        float acc[8];
+        float4 *o = reinterpret_cast<float4 *>(p.out + (size_t)t * p.H) + 2 * k8;
+        if (p.out_add) {
+            const float4 a = o[0], b = o[1];
+            acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+            acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; i++) acc[i] = 0.0f;
+        }
+        float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < NVFP4_MOE_MAX_TOPK; j++) {
+            if (j < p.K) {
+                const __half2 *hv = reinterpret_cast<const __half2 *>(&y[j]);
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const float2 f = __half22float2(hv[i]);
+                    sum[2 * i] += f.x;
+                    sum[2 * i + 1] += f.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; i++) acc[i] += sum[i];
+        o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
 }
 
 // ------------------------------------------------------------------ launch
@@ -244,6 +287,10 @@ void launch_route_large(const Params &p, cudaStream_t s) {
 
 void launch_prep_prefill(const Params &p, cudaStream_t s) {
     prep_prefill_kernel<<<p.T, 256, 0, s>>>(p);
+}
+
+void launch_combine(const Params &p, cudaStream_t s) {
+    combine_kernel<<<p.T, 256, 0, s>>>(p);
 }
 
 
