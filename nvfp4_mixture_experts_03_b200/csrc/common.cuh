@@ -19,9 +19,9 @@ namespace nvmoe {
 constexpr int kChunkTokens = 64;       // tokens per routing CTA (two 32-bit token masks)
 constexpr int kBN = 256;               // max tokens per grouped-GEMM tile (MMA N)
 constexpr int kBK = 64;                // K elements per pipeline stage (one 128B swizzle row)
-constexpr int kGuRows = 64;            // intermediate rows per gate/up tile (64 gate + 64 up)
-constexpr int kDnRows = 128;           // hidden rows per down tile
-constexpr int kStages = 4;             // max smem pipeline depth of the grouped GEMM
+// Grouped-GEMM tiles are computed by a pair of CTAs (one cluster, one M = 256 MMA):
+constexpr int kGuRows = 128;           // intermediates per gate/up tile (64 per CTA: 64 gate + 64 up rows)
+constexpr int kDnRows = 256;           // hidden rows per down tile (128 per CTA; the last may be half)
 
 // Device status block layout (int32 words, 256 bytes): the latched error and its
 // detail, and the decode kernel's grid-wide barrier (generation word, top-level
@@ -120,25 +120,35 @@ __device__ inline void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
         "r"(bytes)
         : "memory");
 }
+template <bool kCluster = false>
 __device__ inline bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
+    if (kCluster)   // arrivals may come from the other CTA of the cluster
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+            " selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+    else
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+            " selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
     return ok != 0;
 }
 // Bounded wait: gives up after `limit_ns` of wall time (or when *abort is set by
 // another thread), latching NVFP4_MOE_ERR_TIMEOUT. Returns false on give-up.
+template <bool kCluster = false>
 __device__ inline bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                  int32_t *status, int where, uint64_t limit_ns = 2000000000ull) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<kCluster>(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     uint32_t spins = 0;
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait<kCluster>(bar, parity)) return true;
         if ((++spins & 63) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > limit_ns) {
@@ -159,6 +169,30 @@ __device__ inline bool mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t 
     return true;
 }
 
+// ------------------------------------------------- clusters of two CTAs
+__device__ inline uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Every thread of every CTA of the cluster (warps must be converged).
+__device__ inline void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ inline uint32_t mapa_shared(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+// Arrive on an mbarrier of any CTA of the cluster (default .release.cta
+// semantics: a cluster-scope release would also wait for this thread's
+// outstanding global loads, i.e. drain the dequant prefetch at every arrival).
+__device__ inline void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 __device__ inline void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -174,6 +208,28 @@ __device__ inline void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
+}
+// Pair form: the box lands in this CTA's shared memory and its bytes are counted
+// on the mbarrier at `bar_cluster` (a shared::cluster address, here the leader
+// CTA's). No multicast.
+__device__ inline void tma_load_2d_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster,
+                                        int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"((uint64_t)map), "r"(bar_cluster), "r"(x), "r"(y)
+        : "memory");
+}
+// 8-byte asynchronous copy global -> shared (both 8-byte aligned).
+__device__ inline void cp_async8(void *dst_smem, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst_smem)), "l"(src)
+                 : "memory");
+}
+// Arrives on `bar` when every cp.async this thread issued so far has landed; the
+// arrival is counted in the barrier's initial count (.noinc).
+__device__ inline void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
 }
 __device__ inline void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
@@ -191,6 +247,19 @@ __device__ inline void tmem_relinquish() {
 __device__ inline void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
 }
+// Pair forms (cta_group::2): one warp with the same warp index in each CTA of the
+// pair issues alloc / relinquish / dealloc; the same columns are taken in both.
+__device__ inline void tmem_alloc_pair(uint32_t *slot_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(slot_smem)),
+                 "r"(ncols));
+}
+__device__ inline void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+}
+__device__ inline void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
 __device__ inline void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -204,6 +273,31 @@ __device__ inline void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdes
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// Pair MMA (issued by the leader CTA only): M = 256 rows, the first 128 from the
+// leader's A tile and TMEM, the next 128 from the peer's; B's first N/2 rows from
+// the leader's shared memory and the other N/2 from the peer's (same offsets).
+__device__ inline void tc_mma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// Arrives on the mbarrier at the same offset in every CTA of `cta_mask` once the
+// pair MMAs issued so far by this thread have completed.
+__device__ inline void tc_commit_pair_mc(uint64_t *bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+__device__ inline void tc_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
 }
 // Arrives on `bar` once every tcgen05.mma issued so far by this thread has completed.
 __device__ inline void tc_commit(uint64_t *bar) {
@@ -280,7 +374,9 @@ __device__ inline void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ inline float silu(float z) { return z / (1.0f + __expf(-z)); }
+// z * sigmoid(z) with the fast exponential and divide intrinsics (relative error
+// a few FP32 ulps; z -> -inf gives exp = inf and a zero quotient).
+__device__ inline float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // Per-token power-of-two factor 2^k with amax * 2^k in [2^14, 2^15): every BF16
 // value within 2^28 of the token's amax is exact in F16 after the shift.
@@ -297,11 +393,19 @@ void launch_route_large(const Params &p, cudaStream_t s);
 void launch_prep_prefill(const Params &p, cudaStream_t s);
 void launch_combine(const Params &p, cudaStream_t s);   // prefill: per-token sum of the K pair rows
 cudaError_t launch_decode(const Params &p, cudaStream_t s);   // the whole T <= 8 layer
-// mode 0: gate/up + SwiGLU, map = F16 activations [P][H]; mode 1: down + combine,
-// map = h [P][I]; both 64 x 64 boxes
-void launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &map, int num_sms,
-                         cudaStream_t s);
-cudaError_t prefill_init();   // per device: opt the GEMM kernels into their shared memory
+// mode 0: gate/up + SwiGLU, map_b = F16 activations [P][H]; mode 1: down, map_b =
+// h [P][I]; both 64 x 64 boxes
+// Tensor maps of the packed E2M1 code planes (bytes; 128-byte x 64-row boxes for
+// gate and up, 128-row boxes for down; 128-byte swizzle).
+struct CodeMaps {
+    CUtensorMap gate, up, down;
+};
+// Clusters of two CTAs, at most `max_clusters` of them (persistent).
+cudaError_t launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &map_b,
+                                const CodeMaps &codes, int max_clusters, cudaStream_t s);
+// Per device: opt the GEMM kernels into their shared memory; *max_clusters = how
+// many CTA pairs of either GEMM can be resident at once.
+cudaError_t prefill_init(int *max_clusters);
 cudaError_t decode_init();    // per device: opt the decode kernels into their shared memory
 
 }  // namespace nvmoe

@@ -23,6 +23,8 @@ struct nvfp4_moe {
     nvfp4_moe_weights w;
     int device;
     int num_sms;
+    int pf_clusters;  // resident CTA pairs of the prefill GEMMs
+    CodeMaps codes;   // tensor maps of the weight code planes (prefill GEMMs)
     int32_t *status;  // kStatusWords ints on the device
     cudaEvent_t phase[NVFP4_MOE_PHASE_EVENTS];
     bool phase_on;
@@ -63,6 +65,21 @@ bool make_map_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Packed E2M1 code plane [rows][cols] bytes: 128-byte x box_rows boxes, swizzled
+// like the GEMM's shared-memory tiles.
+bool make_map_codes(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols};
+    cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 inline bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
@@ -81,7 +98,7 @@ WsLayout layout(const nvfp4_moe_dims &d, int T) {
     const bool decode = T <= NVFP4_MOE_DECODE_MAX_T;
     const size_t ntile_n = P / kBN + (size_t)(E < (int)P ? E : (int)P) + 1;
     L.max_gu = decode ? 0 : (int)(ntile_n * (d.inter / kGuRows));
-    L.max_dn = decode ? 0 : (int)(ntile_n * (d.hidden / kDnRows));
+    L.max_dn = decode ? 0 : (int)(ntile_n * cdiv(d.hidden, kDnRows));
     size_t o = 0;
     auto take = [&](size_t bytes) {
         const size_t at = o;
@@ -162,7 +179,8 @@ int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (major != 10) return NVFP4_MOE_ERR_NO_DEVICE;
-    if (prefill_init() != cudaSuccess || decode_init() != cudaSuccess || !encode_fn())
+    int pf_clusters = 0;
+    if (prefill_init(&pf_clusters) != cudaSuccess || decode_init() != cudaSuccess || !encode_fn())
         return NVFP4_MOE_ERR_CUDA;
     nvfp4_moe *h = new (std::nothrow) nvfp4_moe;
     if (!h) return NVFP4_MOE_ERR_CUDA;
@@ -170,6 +188,14 @@ int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
     h->w = *w;
     h->device = dev;
     h->num_sms = sms;
+    h->pf_clusters = pf_clusters;
+    const int64_t E = d.n_experts;
+    if (!make_map_codes(&h->codes.gate, w->gate_codes, E * d.inter, d.hidden / 2, 64) ||
+        !make_map_codes(&h->codes.up, w->up_codes, E * d.inter, d.hidden / 2, 64) ||
+        !make_map_codes(&h->codes.down, w->down_codes, E * d.hidden, d.inter / 2, 128)) {
+        delete h;
+        return NVFP4_MOE_ERR_CUDA;
+    }
     h->status = nullptr;
     h->phase_on = false;
     if (cudaMalloc(&h->status, kStatusWords * sizeof(int32_t)) != cudaSuccess ||
@@ -296,9 +322,11 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
         mark(1);
         launch_prep_prefill(p, s);
         mark(2);
-        launch_prefill_gemm(0, p, map_xh, h->num_sms, s);
+        if (launch_prefill_gemm(0, p, map_xh, h->codes, h->pf_clusters, s) != cudaSuccess)
+            return NVFP4_MOE_ERR_CUDA;
         mark(3);
-        launch_prefill_gemm(1, p, map_h, h->num_sms, s);
+        if (launch_prefill_gemm(1, p, map_h, h->codes, h->pf_clusters, s) != cudaSuccess)
+            return NVFP4_MOE_ERR_CUDA;
         launch_combine(p, s);
         mark(4);
     }
@@ -427,6 +455,7 @@ int nvfp4_moe_forward_decode_static(const nvfp4_moe_dims *dims, const nvfp4_moe_
     h.w = *w;
     h.device = dev;
     h.num_sms = sms;
+    h.pf_clusters = 0;   // T <= 8 never reaches the prefill GEMMs
     h.status = reinterpret_cast<int32_t *>(scratch);
     h.phase_on = false;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

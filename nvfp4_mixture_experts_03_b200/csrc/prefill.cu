@@ -1,76 +1,94 @@
-// Prefill grouped GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM).
+// Prefill grouped GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM),
+// computed by pairs of CTAs (clusters of two, one M = 256 pair MMA per K step).
 //
-// One persistent CTA per SM walks a device-built tile list (expert, 128 output
+// One persistent CTA pair walks a device-built tile list (expert, 256 output
 // rows, up to 256 token pairs); no host read-back of counts ("Strata NVFP4"
 // README, "How it differs from upstream Strata": one launch per expert group
 // after one wait). Bigger prompt chunks re-stream each expert fewer times
 // ("strata-5090-4070" README, "RAM: the one thing to know"), which is why a tile
 // covers up to 256 pairs of one expert.
 //
-// Operands, per 64-wide K stage:
-//   A (weights, M = 128 rows): dequantised by four warps from the packed planes
-//     straight into the 128-byte-swizzled K-major layout. code x E4M3 scale is
-//     exact in F16, so the MMA sees the stored weights without rounding. The
-//     FP32 tensor scale is applied in the epilogue ("Strata NVFP4" README, "How
-//     it differs": per-expert FP32 scales applied to each projection's output).
-//   B (activations, N = pairs): the F16 copy of x (gate/up) or h (down) rows of
-//     this expert's pairs, brought in by TMA with the same swizzle.
-//   D (FP32, 128 lanes x N columns) in TMEM, double-buffered so the epilogue of
-//     one tile overlaps the MMAs of the next.
-// Epilogues: gate/up -> scales, SwiGLU, F16 h at the pair's position (64 gate
-// rows and 64 up rows of the same intermediate indices share a tile, arranged
-// so that each TMEM lane quarter holds 16 gate and the matching 16 up rows);
+// Operands, per 64-wide K stage, in each CTA of the pair:
+//   A (weights, 128 of the tile's 256 rows): dequantised by eight warps from the
+//     packed planes straight into the 128-byte-swizzled K-major layout. code x
+//     E4M3 scale is exact in F16, so the MMA sees the stored weights without
+//     rounding. The FP32 tensor scale is applied in the epilogue ("Strata NVFP4"
+//     README, "How it differs": per-expert FP32 scales applied to each
+//     projection's output).
+//   B (activations): half of the tile's pair rows (the F16 copy of x for
+//     gate/up, h for down), brought in by TMA with the same swizzle; the bytes
+//     of both halves are counted on the leader CTA's barrier.
+//   D (FP32, this CTA's 128 rows x N columns) in its own TMEM, double-buffered so
+//     the epilogue of one tile overlaps the MMAs of the next.
+// The leader CTA issues the pair MMAs; their completions are multicast to both
+// CTAs. Compared with one CTA per 128-row tile, each SM streams half the B bytes
+// per MMA and the tensor cores read each B row once for 256 weight rows.
+// Epilogues: gate/up -> scales, SwiGLU, F16 h at the pair's position (each CTA
+// owns 64 intermediates: 64 gate rows and the 64 matching up rows, arranged so
+// that each TMEM lane quarter holds 16 gate and the matching 16 up rows);
 // down -> scale x routing weight, F16 row per pair (combined per token by a
 // separate deterministic kernel).
 //
-// Warp roles (320 threads): 0-3 epilogue, 4-7 dequantise A, 8 TMA for B,
-// 9 TMEM allocation + MMA issue. Every mbarrier wait is bounded (2 s); on
-// give-up the CTA latches NVFP4_MOE_ERR_TIMEOUT, drains its own TMA and MMA
-// work (bounded) and frees its TMEM before returning.
+// Warp roles (480 threads per CTA): 0-3 epilogue, 4-11 dequantise A (two warps
+// per row: one for each half of the 64-wide K stage), 12 TMA for B, 13 TMEM
+// allocation (+ MMA issue in the leader), 14 raw weight stages (codes by TMA,
+// scales by cp.async, 4 K steps per stage) so the dequant warps read only
+// shared memory. Every mbarrier wait is bounded
+// (2 s); on give-up the CTA latches NVFP4_MOE_ERR_TIMEOUT, drains what it can,
+// lets in-flight copies land, and both CTAs free their TMEM after a cluster
+// barrier.
 #include "common.cuh"
 
 namespace nvmoe {
 
-constexpr int kThreads = 320;
-constexpr int kBM = 128;
+constexpr int kThreads = 480;
+constexpr int kBM = 128;                       // A rows per CTA (the pair MMA has M = 256)
+constexpr int kGuCta = kGuRows / 2;            // intermediates per CTA in a gate/up tile
+constexpr int kBRows = kBN / 2;                // B rows per CTA
 constexpr int kAStage = kBM * kBK * 2;         // 16 KB
-constexpr int kBStage = kBN * kBK * 2;         // 32 KB
+constexpr int kBStage = kBRows * kBK * 2;      // 16 KB
 constexpr int kBBox = 64;                      // rows per TMA box
+constexpr int kBoxBytes = kBBox * kBK * 2;     // 8 KB
+constexpr int kRing = 4;                       // A/B pipeline stages
+constexpr int kRawSteps = 4;                   // K steps per raw weight stage
+constexpr int kRawStages = 4;                  // 16 K steps of weights in flight: covers HBM latency
+constexpr int kRawCodeBytes = kBM * kRawSteps * 32;   // 128 rows x 128 B of E2M1 codes
+constexpr int kRawScaleBytes = kBM * kRawSteps * 4;   // 128 rows x 16 B of E4M3 scales
+constexpr int kRawBytes = kRawCodeBytes + kRawScaleBytes;
 constexpr int kTmemCols = 512;                 // two 256-column accumulators
-constexpr int kStageBytes = 32 * kBM * 4;      // one epilogue staging buffer: 32 columns x 128 rows x FP32
-// Both GEMMs: a 4-stage ring and one epilogue staging buffer (a 32-column chunk
-// of h, or of the down projection's per-pair F16 rows).
-template <int MODE> struct Cfg {
-    static constexpr int stages = 4;
-    static constexpr int bufs = 1;
-};
-constexpr int kPF = 4;                         // dequant loads in flight (k-steps)
+constexpr int kEpiBytes = 2 * 32 * kBM * 2;    // epilogue staging: 2 x (32 columns x 128 rows x F16)
+constexpr int kColBytes = kBN * 4;            // the tile's per-column factors (FP32)
 constexpr uint64_t kDrainNs = 200000000ull;    // bounded drain on abort
+constexpr uint64_t kSettleNs = 1000000ull;     // lets in-flight copies land after an abort
+constexpr uint16_t kBothCtas = 0x3;
 
 struct __align__(8) Bars {
-    uint64_t a_full[kStages];
-    uint64_t b_full[kStages];
-    uint64_t empty[kStages];
-    uint64_t acc_full[2];
-    uint64_t acc_empty[2];
+    uint64_t a_full[kRing];     // leader: 8 dequant warps x 2 CTAs
+    uint64_t b_full[kRing];     // leader: expect_tx of both halves
+    uint64_t empty[kRing];      // both: the pair MMA's commit
+    uint64_t raw_full[kRawStages];   // code bytes (TMA) + 32 scale-copy lanes
+    uint64_t raw_empty[kRawStages];  // 8 dequant warps
+    uint64_t acc_full[2];       // both: the pair MMA's commit
+    uint64_t acc_empty[2];      // leader: 4 epilogue warps x 2 CTAs
     uint64_t drain;
     uint32_t tmem_slot;
     int abort;
 };
 
-template <int MODE>
 constexpr size_t smem_bytes() {
-    return 1024 + Cfg<MODE>::stages * (kAStage + kBStage) + Cfg<MODE>::bufs * kStageBytes + sizeof(Bars);
+    return 1024 + kRing * (kAStage + kBStage) + kRawStages * kRawBytes + kEpiBytes + kColBytes +
+           sizeof(Bars);
 }
 
-// Iterates (tile, k-step) pairs of this CTA in order.
+// Iterates (tile, k-step) pairs of this CTA pair in order.
 struct Cursor {
-    int tl, kk, nk, ntl;
-    __device__ Cursor(int nk_, int ntiles) : tl(0), kk(0), nk(nk_) {
-        ntl = ntiles > (int)blockIdx.x ? cdiv(ntiles - (int)blockIdx.x, (int)gridDim.x) : 0;
+    int tl, kk, nk, ntl, cid, ncl;
+    __device__ Cursor(int nk_, int ntiles, int cid_, int ncl_)
+        : tl(0), kk(0), nk(nk_), cid(cid_), ncl(ncl_) {
+        ntl = ntiles > cid ? cdiv(ntiles - cid, ncl) : 0;
     }
     __device__ bool valid() const { return tl < ntl; }
-    __device__ int tile() const { return (int)blockIdx.x + tl * (int)gridDim.x; }
+    __device__ int tile() const { return cid + tl * ncl; }
     __device__ void next() {
         if (++kk == nk) { kk = 0; ++tl; }
     }
@@ -85,147 +103,233 @@ struct Ring {
     }
 };
 
+// First weight row of this CTA's 128-row half of tile t (down: the second half of
+// the last tile lies past H when H % 256 == 128; it then reads the first half's
+// rows, in bounds, and its results are dropped).
 template <int MODE>
-__device__ inline void row_source(const Params &p, const Tile &t, int r, const uint8_t *&codes,
-                                  const uint8_t *&scales) {
+__device__ inline int half_row0(const Params &p, const Tile &t, int rank) {
+    if (MODE == 0) return t.expert * p.I + t.m0 + kGuCta * rank;
+    const int m = t.m0 + kBM * rank < p.H ? t.m0 + kBM * rank : t.m0;
+    return t.expert * p.H + m;
+}
+
+// Where A row r (0..127) of the CTA finds its codes and scales in a raw stage.
+// Gate/up: rows 32q + l hold gate (l < 16) or up (l >= 16) of intermediate
+// 16q + (l & 15); the stage holds 64 gate rows, then 64 up rows.
+template <int MODE>
+__device__ inline void raw_row(int r, int &code_off, int &swz, int &scale_off) {
+    int br, srow;
     if (MODE == 0) {
         const int q = r >> 5, l = r & 31;
-        const int i = t.m0 + 16 * q + (l & 15);
-        const size_t row = (size_t)t.expert * p.I + i;
-        codes = (l < 16 ? p.gate_codes : p.up_codes) + row * (p.H / 2);
-        scales = (l < 16 ? p.gate_scales : p.up_scales) + row * (p.H / 16);
+        br = 16 * q + (l & 15);
+        code_off = (l < 16 ? 0 : kRawCodeBytes / 2) + br * 128;
+        srow = l < 16 ? br : 64 + br;
     } else {
-        const size_t row = (size_t)t.expert * p.H + t.m0 + r;
-        codes = p.down_codes + row * (p.I / 2);
-        scales = p.down_scales + row * (p.I / 16);
+        br = r;
+        code_off = r * 128;
+        srow = r;
     }
+    swz = br & 7;                 // 128-byte swizzle of the TMA box: chunk c at c ^ (row & 7)
+    scale_off = kRawCodeBytes + srow * 16;
 }
 
-struct StepData {
-    uint4 c0, c1;
-    uint32_t s;
-};
-
-__device__ inline StepData load_step(const uint8_t *codes, const uint8_t *scales, int kk) {
-    StepData d;
-    const uint4 *cp = reinterpret_cast<const uint4 *>(codes + 32 * kk);
-    d.c0 = __ldg(cp);
-    d.c1 = __ldg(cp + 1);
-    d.s = __ldg(reinterpret_cast<const uint32_t *>(scales + 4 * kk));
-    return d;
-}
-
-// Writes one 128-byte A row (64 F16 weights) in the 128B-swizzled layout.
-__device__ inline void store_row(uint8_t *a_stage, int r, const StepData &d) {
-    const uint32_t w[8] = {d.c0.x, d.c0.y, d.c0.z, d.c0.w, d.c1.x, d.c1.y, d.c1.z, d.c1.w};
+// Writes half `hf` (64 bytes: 32 F16 weights) of A row r in the 128B-swizzled
+// layout from 16 code bytes and the two E4M3 scales of those 32 weights.
+__device__ inline void store_half_row(uint8_t *a_stage, int r, int hf, uint4 c, uint32_t s2) {
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
     uint8_t *row = a_stage + r * 128;
 #pragma unroll
-    for (int j = 0; j < 8; j++) {
-        const uint32_t sc = e4m3_to_f16x2_bcast(d.s >> (8 * (j >> 1)));
+    for (int jj = 0; jj < 4; jj++) {
+        const int j = 4 * hf + jj;   // 16-byte chunk of the row: weights 8j..8j+7
+        const uint32_t sc = e4m3_to_f16x2_bcast(s2 >> (8 * (jj >> 1)));
         uint32_t o0, o1, o2, o3;
-        e2m1x8_to_f16(w[j], o0, o1, o2, o3);
+        e2m1x8_to_f16(w[jj], o0, o1, o2, o3);
         uint4 v = make_uint4(hmul2(o0, sc), hmul2(o1, sc), hmul2(o2, sc), hmul2(o3, sc));
         *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = v;
     }
 }
 
-// Named barrier over the four epilogue warps (ids 0 is __syncthreads).
+// Named barrier over the four epilogue warps (id 0 is __syncthreads).
 __device__ inline void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// The same barrier with an AND over the 128 epilogue threads: every epilogue
+// thread leaves the tile loop together.
+__device__ inline bool epi_all(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n"
+        " selp.u32 %0, 1, 0, q;\n}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const Params p, const __grid_constant__ CUtensorMap map_b) {
+    grouped_gemm_kernel(const Params p, const __grid_constant__ CUtensorMap map_b,
+                        const __grid_constant__ CUtensorMap map_a0,
+                        const __grid_constant__ CUtensorMap map_a1) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     uint8_t *a_base = smem;
-    constexpr int S = Cfg<MODE>::stages, NB = Cfg<MODE>::bufs;
-    uint8_t *b_base = smem + S * kAStage;
-    uint8_t *epi_stage = b_base + S * kBStage;                       // NB x kStageBytes
-    Bars *bars = reinterpret_cast<Bars *>(epi_stage + NB * kStageBytes);
+    uint8_t *b_base = smem + kRing * kAStage;
+    uint8_t *raw_base = b_base + kRing * kBStage;
+    uint8_t *epi_stage = raw_base + kRawStages * kRawBytes;
+    float *colf_s = reinterpret_cast<float *>(epi_stage + kEpiBytes);
+    Bars *bars = reinterpret_cast<Bars *>(epi_stage + kEpiBytes + kColBytes);
     volatile int *abort = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = (int)cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cid = (int)blockIdx.x >> 1, ncl = (int)gridDim.x >> 1;
     const Tile *tiles = MODE == 0 ? p.tiles_gu : p.tiles_dn;
     const int ntiles = p.cnt[MODE == 0 ? kCntTilesGu : kCntTilesDn];
     const int Kdim = MODE == 0 ? p.H : p.I;
     const int nk = Kdim / kBK;
+    const int ntl = ntiles > cid ? cdiv(ntiles - cid, ncl) : 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; s++) {
-            mbar_init(&bars->a_full[s], 128);
+        for (int s = 0; s < kRing; s++) {
+            mbar_init(&bars->a_full[s], 16);
             mbar_init(&bars->b_full[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
         for (int b = 0; b < 2; b++) {
             mbar_init(&bars->acc_full[b], 1);
-            mbar_init(&bars->acc_empty[b], 128);
+            mbar_init(&bars->acc_empty[b], 8);
+        }
+        for (int s = 0; s < kRawStages; s++) {
+            mbar_init(&bars->raw_full[s], 1 + 32);
+            mbar_init(&bars->raw_empty[s], 8);
         }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         fence_barrier_init();
     }
-    if (warp == 9) {
-        tmem_alloc(&bars->tmem_slot, kTmemCols);
-        tmem_relinquish();
+    if (warp == 13) {
+        tmem_alloc_pair(&bars->tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
     }
-    if (warp == 8 && lane == 0) tma_prefetch_desc(&map_b);
+    if (warp == 12 && lane == 0) tma_prefetch_desc(&map_b);
+    if (warp == 14 && lane == 0) {
+        tma_prefetch_desc(&map_a0);
+        if (MODE == 0) tma_prefetch_desc(&map_a1);
+    }
     tc_fence_before();
     __syncthreads();
+    cluster_sync_all();     // both CTAs' barriers initialised and TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = bars->tmem_slot;
 
-    if (warp >= 4 && warp < 8) {
+    if (warp >= 4 && warp < 12) {
         // ------------------------------------------------ dequantise A rows
-        const int r = threadIdx.x - 128;
-        Cursor ld(nk, ntiles), cs(nk, ntiles);
-        Ring<S> ring;
-        StepData q[kPF];
-        int ld_tile = -1;
-        const uint8_t *lcodes = nullptr, *lscales = nullptr;
-#pragma unroll
-        for (int j = 0; j < kPF; j++) {
-            if (ld.valid()) {
-                if (ld.tile() != ld_tile) {
-                    ld_tile = ld.tile();
-                    row_source<MODE>(p, tiles[ld_tile], r, lcodes, lscales);
-                }
-                q[j] = load_step(lcodes, lscales, ld.kk);
-                ld.next();
-            }
-        }
+        // Thread (r, hf) converts half hf of A row r at every K step, reading the
+        // codes and scales of the current raw stage from shared memory.
+        const int r = (threadIdx.x - 128) & (kBM - 1), hf = (threadIdx.x - 128) >> 7;
+        int code_off, swz, scale_off;
+        raw_row<MODE>(r, code_off, swz, scale_off);
+        Ring<kRing> ring;
+        Ring<kRawStages> rr;
+        uint4 s4 = make_uint4(0, 0, 0, 0);
         bool ok = true;
-        while (ok && cs.valid()) {
-#pragma unroll
-            for (int j = 0; j < kPF; j++) {
-                if (!ok || !cs.valid()) break;
-                if (!mbar_wait(&bars->empty[ring.stage], ring.phase ^ 1, abort, p.status, 1)) {
+        for (int tl = 0; ok && tl < ntl; tl++) {
+            for (int kk = 0; kk < nk; kk++) {
+                const int kq = kk % kRawSteps;
+                const uint8_t *raw = raw_base + rr.stage * kRawBytes;
+                if (kq == 0) {
+                    const bool g = mbar_wait(&bars->raw_full[rr.stage], rr.phase, abort, p.status, 9);
+                    if (!__all_sync(0xffffffffu, g)) {
+                        ok = false;
+                        break;
+                    }
+                    s4 = *reinterpret_cast<const uint4 *>(raw + scale_off);
+                }
+                const bool got = mbar_wait(&bars->empty[ring.stage], ring.phase ^ 1, abort, p.status, 1);
+                if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
                     break;
                 }
-                store_row(a_base + ring.stage * kAStage, r, q[j]);
+                const int c = 2 * kq + hf;
+                const uint4 code = *reinterpret_cast<const uint4 *>(raw + code_off + ((c ^ swz) << 4));
+                const uint32_t sw = kq == 0 ? s4.x : kq == 1 ? s4.y : kq == 2 ? s4.z : s4.w;
+                store_half_row(a_base + ring.stage * kAStage, r, hf, code, sw >> (16 * hf));
                 fence_proxy_async_smem();
-                mbar_arrive(&bars->a_full[ring.stage]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(&bars->a_full[ring.stage], 0));
                 ring.next();
-                cs.next();
-                if (ld.valid()) {
-                    if (ld.tile() != ld_tile) {
-                        ld_tile = ld.tile();
-                        row_source<MODE>(p, tiles[ld_tile], r, lcodes, lscales);
-                    }
-                    q[j] = load_step(lcodes, lscales, ld.kk);
-                    ld.next();
+                if (kq == kRawSteps - 1 || kk == nk - 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->raw_empty[rr.stage]);
+                    rr.next();
                 }
             }
         }
-    } else if (warp == 8) {
+    } else if (warp == 14) {
+        // ------------------------------------------- raw weight stages (A)
+        // Per tile and 4 K steps: the codes of this CTA's 128 rows by TMA (one
+        // 64-row box per gate and up plane, or one 128-row box of down), the
+        // scales by 8-byte copies from all 32 lanes (a scale row's stride need
+        // not be a multiple of 16 bytes, which a tensor map would require).
+        const int kd16 = Kdim / 16;   // scale bytes per weight row
+        Ring<kRawStages> rr;
+        uint32_t issued = 0, issued_phase = 0;
+        bool ok = true;
+        for (int tl = 0; ok && tl < ntl; tl++) {
+            const Tile t = tiles[cid + tl * ncl];
+            const int row0 = half_row0<MODE>(p, t, rank);
+            const uint8_t *sc0 = (MODE == 0 ? p.gate_scales : p.down_scales) + (size_t)row0 * kd16;
+            const uint8_t *sc1 = MODE == 0 ? p.up_scales + (size_t)row0 * kd16 : nullptr;
+            for (int R = 0; R < cdiv(nk, kRawSteps); R++) {
+                const bool g = mbar_wait(&bars->raw_empty[rr.stage], rr.phase ^ 1, abort, p.status, 10);
+                if (!__all_sync(0xffffffffu, g)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *raw = raw_base + rr.stage * kRawBytes;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&bars->raw_full[rr.stage], kRawCodeBytes);
+                    if (MODE == 0) {
+                        tma_load_2d(raw, &map_a0, &bars->raw_full[rr.stage], 128 * R, row0);
+                        tma_load_2d(raw + kRawCodeBytes / 2, &map_a1, &bars->raw_full[rr.stage], 128 * R, row0);
+                    } else {
+                        tma_load_2d(raw, &map_a0, &bars->raw_full[rr.stage], 128 * R, row0);
+                    }
+                    issued |= 1u << rr.stage;
+                    issued_phase = (issued_phase & ~(1u << rr.stage)) | (rr.phase << rr.stage);
+                }
+                // 128 rows x two 8-byte pieces; pieces past the row's end are skipped
+#pragma unroll
+                for (int k = 0; k < (2 * kBM) / 32; k++) {
+                    const int ci = lane + 32 * k, row = ci >> 1, off = 16 * R + 8 * (ci & 1);
+                    if (off < kd16) {
+                        const uint8_t *src = MODE == 0 ? (row < 64 ? sc0 + (size_t)row * kd16
+                                                                   : sc1 + (size_t)(row - 64) * kd16)
+                                                       : sc0 + (size_t)row * kd16;
+                        cp_async8(raw + kRawCodeBytes + row * 16 + 8 * (ci & 1), src + off);
+                    }
+                }
+                cp_async_arrive_noinc(&bars->raw_full[rr.stage]);
+                rr.next();
+            }
+        }
+        // Every raw stage this warp filled must have landed before exit.
+        if (lane == 0)
+            for (int s = 0; s < kRawStages; s++)
+                if (issued & (1u << s))
+                    mbar_wait_drain(&bars->raw_full[s], (issued_phase >> s) & 1, kDrainNs);
+        __syncwarp();
+    } else if (warp == 12) {
         // ------------------------------------------------------ TMA for B
-        // 64-row boxes of the pair-ordered B rows (F16 activations or h) into the
-        // ring; the next tile's descriptor is read one tile ahead.
+        // This CTA's half of the tile's pair rows, in 64-row boxes; the bytes are
+        // counted on the leader's b_full, whose single arrival (with the byte
+        // count of both halves) the leader makes. The next tile's descriptor is
+        // read one tile ahead.
         if (lane == 0) {
-            Cursor cs(nk, ntiles);
-            Ring<S> ring;
-            uint32_t issued = 0, issued_phase = 0;  // stages with a load in flight, their parity
+            Cursor cs(nk, ntiles, cid, ncl);
+            Ring<kRing> ring;
+            uint32_t issued = 0, issued_phase = 0;  // leader: stages with a load in flight
             int cur_tile = -1;
             Tile t{}, t_n{};
             if (cs.valid()) t_n = tiles[cs.tile()];
@@ -233,39 +337,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (cs.tile() != cur_tile) {
                     cur_tile = cs.tile();
                     t = t_n;
-                    if (cur_tile + (int)gridDim.x < ntiles) t_n = tiles[cur_tile + (int)gridDim.x];
+                    if (cur_tile + ncl < ntiles) t_n = tiles[cur_tile + ncl];
                 }
                 if (!mbar_wait(&bars->empty[ring.stage], ring.phase ^ 1, abort, p.status, 2)) break;
-                const int nbox = cdiv((t.ntok + 15) & ~15, kBBox);
+                const int half = ((t.ntok + 15) & ~15) >> 1;
+                const int nbox = cdiv(half, kBBox);
                 uint8_t *bs = b_base + ring.stage * kBStage;
-                mbar_arrive_expect_tx(&bars->b_full[ring.stage], nbox * kBBox * kBK * 2);
+                if (leader) {
+                    mbar_arrive_expect_tx(&bars->b_full[ring.stage], 2 * nbox * kBoxBytes);
+                    issued |= 1u << ring.stage;
+                    issued_phase = (issued_phase & ~(1u << ring.stage)) | (ring.phase << ring.stage);
+                }
+                const uint32_t bar = mapa_shared(&bars->b_full[ring.stage], 0);
                 for (int b = 0; b < nbox; b++)
-                    tma_load_2d(bs + b * kBBox * kBK * 2, &map_b, &bars->b_full[ring.stage],
-                                cs.kk * kBK, t.pos0 + b * kBBox);
-                issued |= 1u << ring.stage;
-                issued_phase = (issued_phase & ~(1u << ring.stage)) | (ring.phase << ring.stage);
+                    tma_load_2d_pair(bs + b * kBoxBytes, &map_b, bar, cs.kk * kBK,
+                                     t.pos0 + rank * half + b * kBBox);
                 ring.next();
                 cs.next();
             }
-            // Every stage's last load must have landed before this CTA may exit.
-            for (int s = 0; s < S; s++)
+            // The leader's last load of every stage must have landed before exit.
+            for (int s = 0; s < kRing; s++)
                 if (issued & (1u << s))
                     mbar_wait_drain(&bars->b_full[s], (issued_phase >> s) & 1, kDrainNs);
         }
-    } else if (warp == 9) {
-        // ----------------------------------------------------- MMA issue
-        if (lane == 0) {
-            Ring<S> ring;
-            uint32_t acc_phase[2] = {0, 0};
-            const int ntl = ntiles > (int)blockIdx.x ? cdiv(ntiles - (int)blockIdx.x, (int)gridDim.x) : 0;
+    } else if (warp == 13) {
+        // ---------------------------------------------- pair MMA issue (leader)
+        if (leader && lane == 0) {
+            Ring<kRing> ring;
+            uint32_t acc_phase = 0;     // bit b: parity of accumulator b's next use
             bool ok = true;
             for (int tl = 0; ok && tl < ntl; tl++) {
-                const Tile t = tiles[(int)blockIdx.x + tl * (int)gridDim.x];
+                const Tile t = tiles[cid + tl * ncl];
                 const int buf = tl & 1;
                 const int nmma = (t.ntok + 15) & ~15;
-                const uint32_t idesc = idesc_f16(kBM, nmma);
-                if (!mbar_wait(&bars->acc_empty[buf], acc_phase[buf] ^ 1, abort, p.status, 4)) break;
-                acc_phase[buf] ^= 1;
+                const uint32_t idesc = idesc_f16(2 * kBM, nmma);
+                if (!mbar_wait(&bars->acc_empty[buf], ((acc_phase >> buf) & 1) ^ 1, abort, p.status, 4))
+                    break;
+                acc_phase ^= 1u << buf;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * kBN;
                 for (int kk = 0; kk < nk; kk++) {
@@ -279,40 +387,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t bs = smem_u32(b_base + ring.stage * kBStage);
 #pragma unroll
                     for (int k16 = 0; k16 < kBK / 16; k16++)
-                        tc_mma_f16(d_tmem, smem_desc_sw128(as + 32 * k16),
-                                   smem_desc_sw128(bs + 32 * k16), idesc, (kk | k16) != 0);
-                    tc_commit(&bars->empty[ring.stage]);
+                        tc_mma_f16_pair(d_tmem, smem_desc_sw128(as + 32 * k16),
+                                        smem_desc_sw128(bs + 32 * k16), idesc, (kk | k16) != 0);
+                    tc_commit_pair_mc(&bars->empty[ring.stage], kBothCtas);
                     ring.next();
                 }
-                if (ok) tc_commit(&bars->acc_full[buf]);
+                if (ok) tc_commit_pair_mc(&bars->acc_full[buf], kBothCtas);
             }
             // Drain: every MMA this thread issued completes before TMEM is freed.
-            tc_commit(&bars->drain);
+            tc_commit_pair(&bars->drain);
             mbar_wait_drain(&bars->drain, 0, kDrainNs);
         }
     } else {
         // -------------------------------------------------------- epilogue
-        const int ntl = ntiles > (int)blockIdx.x ? cdiv(ntiles - (int)blockIdx.x, (int)gridDim.x) : 0;
-        uint32_t acc_phase[2] = {0, 0};
+        // Per tile: the tile's per-column factors (activation scale, or routing
+        // weight x s_d) are loaded before the accumulator wait and parked in
+        // shared memory; each 32-column chunk is staged in shared memory (two
+        // buffers, one named barrier per chunk) and written with coalesced 16-byte
+        // stores.
+        constexpr int kChunks = kBN / 32;
+        uint32_t acc_phase = 0;
         for (int tl = 0; tl < ntl; tl++) {
-            const Tile t = tiles[(int)blockIdx.x + tl * (int)gridDim.x];
+            const Tile t = tiles[cid + tl * ncl];
             const int buf = tl & 1;
-            if (!mbar_wait(&bars->acc_full[buf], acc_phase[buf], abort, p.status, 8)) break;
-            acc_phase[buf] ^= 1;
+            const int e = t.expert;
+            const float *colf = MODE == 0 ? p.ps : p.pw;
+            const float cscale = MODE == 0 ? 1.0f : p.down_global[e];
+            float cf[kBN / 128];
+#pragma unroll
+            for (int c = 0; c < kBN / 128; c++) {
+                const int col = 128 * c + threadIdx.x;
+                cf[c] = col < t.ntok ? colf[t.pos0 + col] * cscale : 0.0f;
+            }
+            const bool got = mbar_wait(&bars->acc_full[buf], (acc_phase >> buf) & 1, abort, p.status, 8);
+            // The AND-barrier also orders every read of colf_s for the previous
+            // tile before the writes below.
+            if (!epi_all(got)) break;
+#pragma unroll
+            for (int c = 0; c < kBN / 128; c++) colf_s[128 * c + threadIdx.x] = cf[c];
+            epi_sync();
+            acc_phase ^= 1u << buf;
             tc_fence_after();
             const uint32_t tbase = tmem_base + buf * kBN + ((uint32_t)(warp * 32) << 16);
-            const int e = t.expert;
             if (MODE == 0) {
-                // SwiGLU; h staged as [32 columns][64 intermediates] F16, then written
-                // with coalesced 16-byte stores (each column is 128 contiguous bytes of h).
+                // SwiGLU; h staged as [32 columns][64 intermediates] F16 (each column
+                // is 128 contiguous bytes of h).
                 const float sg = p.gate_global[e], su = p.up_global[e];
                 const int il = 16 * warp + (lane & 15);
                 const bool is_gate = lane < 16;
-                __half *hs = reinterpret_cast<__half *>(epi_stage);
-                for (int c0 = 0; c0 < t.ntok; c0 += 32) {
+                const int i0 = t.m0 + kGuCta * rank;
+#pragma unroll 1
+                for (int c = 0; c < kChunks; c++) {
+                    if (32 * c >= t.ntok) break;
+                    __half *hs = reinterpret_cast<__half *>(epi_stage) + (c & 1) * (32 * kGuCta);
                     uint32_t v[32];
-                    tmem_ld32(tbase + c0, v);
-                    const float xs_l = (c0 + lane < t.ntok) ? p.ps[t.pos0 + c0 + lane] : 0.0f;
+                    tmem_ld32(tbase + 32 * c, v);
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
@@ -323,71 +452,107 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float gacc = is_gate ? mine_lo : recv;
                         const float uacc = is_gate ? recv : mine_hi;
                         const int cj = j + (is_gate ? 0 : 16);
-                        const float xs = __shfl_sync(0xffffffffu, xs_l, cj);
+                        const float xs = colf_s[32 * c + cj];
                         const float gv = gacc * sg * xs, uv = uacc * su * xs;
-                        hs[cj * kGuRows + il] = __float2half_rn(silu(gv) * uv);
+                        hs[cj * kGuCta + il] = __float2half_rn(silu(gv) * uv);
                     }
                     epi_sync();
-                    const int ncol = min(32, t.ntok - c0);
-                    for (int q = threadIdx.x; q < ncol * 8; q += 128) {
-                        const int col = q >> 3, part = q & 7;
-                        const uint4 val = reinterpret_cast<const uint4 *>(hs + col * kGuRows)[part];
-                        reinterpret_cast<uint4 *>(p.h + (size_t)(t.pos0 + c0 + col) * p.I + t.m0)[part] = val;
+                    const int ncol = min(32, t.ntok - 32 * c);
+                    for (int q = threadIdx.x; q < ncol * (kGuCta / 8); q += 128) {
+                        const int col = q / (kGuCta / 8), part = q % (kGuCta / 8);
+                        const uint4 val = reinterpret_cast<const uint4 *>(hs + col * kGuCta)[part];
+                        reinterpret_cast<uint4 *>(p.h + (size_t)(t.pos0 + 32 * c + col) * p.I + i0)[part] = val;
                     }
-                    epi_sync();
                 }
             } else {
-                // y * s_d * w staged as [32 columns][128 hidden rows] F16, written with
-                // coalesced 16-byte stores into the pair's row of yp; the combine
-                // kernel sums each token's K rows in a fixed order.
-                const float sd = p.down_global[e];
+                // y * s_d * w staged as [32 columns][128 hidden rows] F16, written into
+                // the pair's row of yp; the combine kernel sums each token's K rows in
+                // a fixed order.
                 const int r = 32 * warp + lane;
-                __half *ys = reinterpret_cast<__half *>(epi_stage);
-                for (int c0 = 0; c0 < t.ntok; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(tbase + c0, v);
-                    const float w_l = (c0 + lane < t.ntok) ? p.pw[t.pos0 + c0 + lane] * sd : 0.0f;
-                    tmem_ld_wait();
+                const int m = t.m0 + kBM * rank;
+                if (m < p.H) {
+#pragma unroll 1
+                    for (int c = 0; c < kChunks; c++) {
+                        if (32 * c >= t.ntok) break;
+                        __half *ys = reinterpret_cast<__half *>(epi_stage) + (c & 1) * (32 * kBM);
+                        uint32_t v[32];
+                        tmem_ld32(tbase + 32 * c, v);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; j++)
-                        ys[j * kBM + r] = __float2half_rn(__uint_as_float(v[j]) * __shfl_sync(0xffffffffu, w_l, j));
-                    epi_sync();
-                    const int ncol = min(32, t.ntok - c0);
-                    for (int q = threadIdx.x; q < ncol * (kBM / 8); q += 128) {
-                        const int col = q / (kBM / 8), part = q % (kBM / 8);
-                        const uint4 val = reinterpret_cast<const uint4 *>(ys + col * kBM)[part];
-                        reinterpret_cast<uint4 *>(p.xh + (size_t)(t.pos0 + c0 + col) * p.H + t.m0)[part] = val;
+                        for (int j = 0; j < 32; j++)
+                            ys[j * kBM + r] = __float2half_rn(__uint_as_float(v[j]) * colf_s[32 * c + j]);
+                        epi_sync();
+                        const int ncol = min(32, t.ntok - 32 * c);
+                        for (int q = threadIdx.x; q < ncol * (kBM / 8); q += 128) {
+                            const int col = q / (kBM / 8), part = q % (kBM / 8);
+                            const uint4 val = reinterpret_cast<const uint4 *>(ys + col * kBM)[part];
+                            reinterpret_cast<uint4 *>(p.xh + (size_t)(t.pos0 + 32 * c + col) * p.H + m)[part] = val;
+                        }
                     }
-                    epi_sync();
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars->acc_empty[buf]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(&bars->acc_empty[buf], 0));
         }
     }
 
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (threadIdx.x == 0 && *abort) {
+        // After a give-up, copies this CTA started may still be landing in its
+        // shared memory (the peer's loads are counted on the leader's barrier).
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < kSettleNs) __nanosleep(1000);
+    }
+    __syncthreads();
+    cluster_sync_all();     // no pair MMA, copy or remote arrive touches either CTA past here
+    if (warp == 13) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 }
 
-cudaError_t prefill_init() {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<0>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes<0>());
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_bytes<1>());
+static cudaLaunchConfig_t gemm_config(int nclusters, cudaStream_t s, cudaLaunchAttribute *attr) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * nclusters);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem_bytes();
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
 }
 
-void launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &map, int num_sms,
-                         cudaStream_t s) {
-    if (mode == 0)
-        grouped_gemm_kernel<0><<<max(1, min(num_sms, p.max_tiles_gu)), kThreads, smem_bytes<0>(), s>>>(p, map);
-    else
-        grouped_gemm_kernel<1><<<max(1, min(num_sms, p.max_tiles_dn)), kThreads, smem_bytes<1>(), s>>>(p, map);
+cudaError_t prefill_init(int *max_clusters) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<0>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes());
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem_bytes());
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = gemm_config(1, 0, attr);
+    int n0 = 0, n1 = 0;
+    e = cudaOccupancyMaxActiveClusters(&n0, grouped_gemm_kernel<0>, &cfg);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n1, grouped_gemm_kernel<1>, &cfg);
+    if (e != cudaSuccess) return e;
+    *max_clusters = n0 < n1 ? n0 : n1;
+    return *max_clusters > 0 ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+cudaError_t launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &map_b,
+                                const CodeMaps &codes, int max_clusters, cudaStream_t s) {
+    const int maxt = mode == 0 ? p.max_tiles_gu : p.max_tiles_dn;
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = gemm_config(max(1, min(max_clusters, maxt)), s, attr);
+    return mode == 0 ? cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<0>, p, map_b, codes.gate, codes.up)
+                     : cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<1>, p, map_b, codes.down, codes.down);
 }
 
 }  // namespace nvmoe

@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(Params p) {
     int *wt = dnb + p.E;                  // [33]
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) cnt_s[e] = p.counts[e];
     __syncthreads();
-    const int mgu = p.I / kGuRows, mdn = p.H / kDnRows;
+    const int mgu = p.I / kGuRows, mdn = cdiv(p.H, kDnRows);
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
         off_s[e] = cnt_s[e];
         gub[e] = cdiv(cnt_s[e], kBN) * mgu;

@@ -82,6 +82,18 @@ def test_medium_skewed_multi_tile(T):
     assert_close(out, ref["out"], f"medium T={T}")
 
 
+@pytest.mark.parametrize("T", [3, 260])
+def test_hidden_not_multiple_of_256(T):
+    """H = 384: the down projection's last 256-row tile is half past H (its second
+    CTA computes nothing that is kept); I = 128 is a single gate/up tile."""
+    dims = synth.LayerDims(E=12, H=384, I=128, K=3)
+    layer, logits, x, xs = _case(dims, T, seed=57, zipf=0.8)
+    ref, out, dbg, st = _run_both(layer, logits, x, xs, dims.K)
+    assert st == 0
+    check_routing(dbg, ref, T, dims.K)
+    assert_close(out, ref["out"], f"H=384 T={T}")
+
+
 def test_one_expert_takes_every_token_and_k_equals_e():
     dims = synth.LayerDims(E=8, H=256, I=128, K=8)
     T = 40
