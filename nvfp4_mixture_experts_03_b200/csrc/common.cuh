@@ -31,6 +31,11 @@ enum : int { kStatusCode = 0, kStatusDetail = 1, kStatusBarGen = 8, kStatusBarTo
 
 // Per-call routing/tile counters kept in the workspace (int32 words).
 enum : int { kCntTilesGu = 0, kCntTilesDn = 1, kCntUniq = 2, kCntWords = 64 };
+// Decode state (per handle, zero between launches): int words, then the FP32
+// gate/up partial sums [pairs][2][I]. kDsStaged: CTAs past their activation
+// reads; kDsExit: CTAs done; kDsReady + u: finished gate/up items of used
+// expert u; kDsItems + item: K rounds summed so far of a split gate/up item.
+enum : int { kDsStaged = 0, kDsExit = 1, kDsReady = 2, kDsItems = 2 + 128 };
 
 struct Tile {  // one grouped-GEMM tile
     int32_t expert;   // expert id
@@ -82,6 +87,9 @@ struct Params {
     int32_t *dbg_counts, *dbg_offsets, *dbg_perm;
     int32_t nch;               // routing chunks
     int32_t max_tiles_gu, max_tiles_dn;
+    int32_t *dstate;           // decode: counters (kDs*), zero between launches
+    float *dgu;                // decode: [pairs][2][I] FP32 partial sums, zero between launches
+    int32_t dec_hs_rows;       // decode: h rows one CTA stages for its down range
 };
 
 constexpr int kActF32 = 2;     // internal: act is FP32, rounded to BF16 first
@@ -393,6 +401,15 @@ void launch_route_large(const Params &p, cudaStream_t s);
 void launch_prep_prefill(const Params &p, cudaStream_t s);
 void launch_combine(const Params &p, cudaStream_t s);   // prefill: per-token sum of the K pair rows
 cudaError_t launch_decode(const Params &p, cudaStream_t s);   // the whole T <= 8 layer
+int decode_grid();                                 // CTAs of the decode kernel (one per SM)
+int decode_hs_rows(int T, int K, int E, int grid); // h rows one decode CTA may stage
+// Bytes of the decode state for up to `pairs` (token, slot) pairs.
+inline size_t decode_state_ints_bytes(int pairs, int inter) {
+    return (((size_t)kDsItems + (size_t)pairs * (inter / 8)) * 4 + 255) & ~size_t(255);
+}
+inline size_t decode_state_bytes(int pairs, int inter) {
+    return decode_state_ints_bytes(pairs, inter) + (size_t)pairs * 2 * inter * 4;
+}
 // mode 0: gate/up + SwiGLU, map_b = F16 activations [P][H]; mode 1: down, map_b =
 // h [P][I]; both 64 x 64 boxes
 // Tensor maps of the packed E2M1 code planes (bytes; 128-byte x 64-row boxes for

@@ -5,17 +5,28 @@
 // the measurements) and note that a decode round is bound by moving expert
 // bytes ("Strata NVFP4" README, "Limits"). On B200 every expert is resident in
 // HBM, so decode is a pure HBM stream whose time is set by how early the weight
-// loads start and how many are in flight.
+// loads start, how many are in flight, and how evenly the bytes are spread.
 //
-// Two kernels, linked by programmatic dependent launch:
-//   gate/up: waits for the previous grid (griddepcontrol.wait), then every CTA
-//     routes the <= 8 tokens itself (top-k over at most 8 x E logits is a few
-//     microseconds of one warp per token), so it knows the selected experts
-//     without another kernel or a grid-wide barrier, and starts its weight stream.
-//   down: launched as soon as every gate/up CTA has passed its wait; routes again
-//     in every CTA, issues its first weight loads, and only then waits for the
-//     gate/up grid (whose h it needs), so its weight stream overlaps the gate/up
-//     kernel.
+// One kernel per layer, one 16-warp CTA per SM, launched with programmatic
+// dependent launch (each CTA lets the next layer's grid launch once its own work
+// is done):
+//   routing: every CTA routes the <= 8 tokens itself (warp top-k per token, then
+//     the <= 128 (token, slot) pairs ranked by (expert, token) to give positions,
+//     the used-expert list and each (expert, token) position and weight);
+//   phase 1 (gate/up + SwiGLU): the units (used expert, 8 intermediates, 128-wide
+//     K round) are cut into equal contiguous ranges, one per warp of the grid.
+//     A warp that covers a whole item applies SwiGLU to its registers; partial
+//     items add their FP32 sums into a per-handle accumulator, and the warp whose
+//     contribution completes the item applies SwiGLU from there (clearing it).
+//     Every finished item counts towards its expert's ready count;
+//   phase 2 (down + weighted combine): the units (used expert, 16 hidden rows,
+//     128-wide K round) are cut into equal contiguous ranges, one per CTA (split
+//     evenly over its warps). A CTA issues its first weight loads, waits only for
+//     the ready counts of the one or two experts its range touches, copies their
+//     h rows into shared memory, and adds its partial sums into out.
+// No grid-wide barrier: the only cross-CTA waits are the per-expert ready counts
+// and one count of CTAs that have read the activations (out may alias them),
+// all bounded. The last CTA to finish resets the counts for the next launch.
 // Arithmetic: each weight is decoded exactly to F16 (E2M1 -> F16 conversion
 // times its E4M3 group scale: at most 6 significant bits, exact in F16) and fed
 // to mma.sync m16n8k16 with the token slots as N, FP32 accumulation; the tensor
@@ -65,42 +76,35 @@ __device__ inline void round_mma(float (&acc)[4], const uint4 &ca, const uint4 &
     }
 }
 
-constexpr int kDecWarps = 8;
+
+constexpr int kDecWarps = 16;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kMaxRoundsPerWarp = 4;   // 128-wide K rounds of loads one warp holds per pass
-constexpr int kMaxUniq = NVFP4_MOE_DECODE_MAX_T * NVFP4_MOE_MAX_TOPK;  // 128
+constexpr int kMaxRoundsPerWarp = 4;   // 128-wide K rounds of loads one warp holds per chunk
+constexpr int kMaxPairs = NVFP4_MOE_DECODE_MAX_T * NVFP4_MOE_MAX_TOPK;  // 128
 constexpr int kSlots = NVFP4_MOE_DECODE_MAX_T;
+constexpr uint64_t kDecWaitNs = 200000000ull;
 
-// Number of warps that share one item's K range (1, 2 or 4): each warp takes
-// rounds/split consecutive rounds; the partial sums meet in shared memory.
-__host__ __device__ inline int k_split(int rounds) {
-    if (rounds % 4 == 0 && rounds / 4 <= kMaxRoundsPerWarp) return 4;
-    if (rounds % 2 == 0 && rounds / 2 <= kMaxRoundsPerWarp) return 2;
-    return rounds <= kMaxRoundsPerWarp ? 1 : 4;
-}
-
-// Per-CTA routing state of the decode kernels.
+// Per-CTA routing state of the decode kernel.
 struct DecRoute {
-    int ids[kSlots * NVFP4_MOE_MAX_TOPK];
-    float w[kSlots * NVFP4_MOE_MAX_TOPK];
-    int uniq[kMaxUniq];             // selected experts, ascending
-    int upos[kMaxUniq * kSlots];    // pair position of (unique expert, token), -1 if absent
-    float uw[kMaxUniq * kSlots];    // routing weight of (unique expert, token)
+    int ids[kMaxPairs];
+    float w[kMaxPairs];
+    int pos[kMaxPairs];             // position of pair q (grouped by expert, then token)
+    int sorted_e[kMaxPairs];        // expert at each position
+    int uniq[kMaxPairs];            // used experts, ascending
+    int uoff[kMaxPairs + 1];        // first position of each used expert; uoff[U] = P
+    int upos[kMaxPairs * kSlots];   // pair position of (used expert, token), -1 if absent
+    float uw[kMaxPairs * kSlots];   // routing weight of (used expert, token)
     unsigned amax[kSlots];          // per-token activation amax (FP32 bits)
     float xsc[kSlots];              // per-token factor that undoes the F16 staging scale
-    int U, total;
-    int wt[33];
+    int U;
 };
 
-// Routes the T <= 8 tokens inside one CTA (identical result in every CTA):
-// top-k + weights, per-expert token masks, counts and offsets by one packed
-// scan, the unique-expert list and each (expert, token) position and weight.
-// emask/cnt: E ints each of dynamic shared memory.
+// Routes the T <= 8 tokens inside one CTA (identical result in every CTA).
 template <int NPER>
-__device__ void cta_route(const Params &p, DecRoute &R, int *emask, int *cnt, bool report) {
+__device__ void cta_route(const Params &p, DecRoute &R, bool report) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int e = threadIdx.x; e < p.E; e += blockDim.x) emask[e] = 0;
-    __syncthreads();
+    const int P = p.T * p.K;
+    for (int i = threadIdx.x; i < kMaxPairs * kSlots; i += blockDim.x) R.upos[i] = -1;
     if (warp < p.T) {
         int id;
         float w;
@@ -116,57 +120,75 @@ __device__ void cta_route(const Params &p, DecRoute &R, int *emask, int *cnt, bo
         if (lane < p.K) {
             R.ids[warp * p.K + lane] = id;
             R.w[warp * p.K + lane] = w;
-            atomicOr(&emask[id], 1 << warp);
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
-        const int c = __popc(emask[e]);
-        cnt[e] = c | ((c != 0) << 16);   // pairs (low 16 bits), used experts (high 16 bits)
+    // A token's ids are distinct, so ordering the pairs q = t*K + j by (expert, q)
+    // groups them by expert and, within an expert, by token.
+    const int q = threadIdx.x;
+    int e = 0, rank = 0;
+    if (q < P) {
+        e = R.ids[q];
+        const int key = (e << 7) | q;
+        for (int j = 0; j < P; j++) rank += ((R.ids[j] << 7) | j) < key;
+        R.pos[q] = rank;
+        R.sorted_e[rank] = e;
     }
     __syncthreads();
-    const int both = block_exscan(cnt, p.E, R.wt);
+    const bool first = q < P && (rank == 0 || R.sorted_e[rank - 1] != e);
+    const int U = __syncthreads_count(first);
+    if (first) {
+        int u = 0;   // distinct experts at positions before this one
+        for (int j = 1; j < rank; j++) u += R.sorted_e[j] != R.sorted_e[j - 1];
+        u += rank > 0;
+        R.uniq[u] = e;
+        R.uoff[u] = rank;
+    }
     if (threadIdx.x == 0) {
-        R.total = both & 0xFFFF;
-        R.U = both >> 16;
+        R.U = U;
+        R.uoff[U] = P;
     }
-    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
-        if (emask[e]) R.uniq[cnt[e] >> 16] = e;
-    for (int i = threadIdx.x; i < kMaxUniq * kSlots; i += blockDim.x) R.upos[i] = -1;
     __syncthreads();
-    for (int q = threadIdx.x; q < p.T * p.K; q += blockDim.x) {   // one thread per (token, slot)
-        const int t = q / p.K, e = R.ids[q];
-        const int u = cnt[e] >> 16;
-        R.upos[u * kSlots + t] = (cnt[e] & 0xFFFF) + __popc(emask[e] & ((1 << t) - 1));
-        R.uw[u * kSlots + t] = R.w[q];
+    if (q < P) {
+        int lo = 0, hi = U - 1;   // u of this pair's expert (uniq ascending)
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (R.uniq[mid] <= e) lo = mid; else hi = mid - 1;
+        }
+        const int t = q / p.K;
+        R.upos[lo * kSlots + t] = rank;
+        R.uw[lo * kSlots + t] = R.w[q];
     }
     __syncthreads();
 }
 
 // The routing results a forward call leaves in the workspace (and the optional
-// debug copies); written by CTA 0 after the previous grid has finished.
-__device__ void publish_route(const Params &p, const DecRoute &R, const int *emask, const int *cnt) {
-    for (int q = threadIdx.x; q < p.T * p.K; q += blockDim.x) {
-        const int t = q / p.K, e = R.ids[q];
-        const int pos = (cnt[e] & 0xFFFF) + __popc(emask[e] & ((1 << t) - 1));
-        p.ids[q] = e;
+// debug copies); written by CTA 0.
+__device__ void publish_route(const Params &p, const DecRoute &R) {
+    const int P = p.T * p.K;
+    for (int q = threadIdx.x; q < P; q += blockDim.x) {
+        const int pos = R.pos[q], t = q / p.K;
+        p.ids[q] = R.ids[q];
         p.wts[q] = R.w[q];
         p.perm[pos] = q;
         p.inv[q] = pos;
         p.ptok[pos] = t;
         p.pw[pos] = R.w[q];
-        if (p.dbg_ids) p.dbg_ids[q] = e;
+        if (p.dbg_ids) p.dbg_ids[q] = R.ids[q];
         if (p.dbg_w) p.dbg_w[q] = R.w[q];
         if (p.dbg_perm) p.dbg_perm[pos] = q;
     }
     for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
-        const int off = e < p.E ? (cnt[e] & 0xFFFF) : R.total;
-        p.offsets[e] = off;
-        if (p.dbg_offsets) p.dbg_offsets[e] = off;
+        int before = 0, at = 0;
+        for (int j = 0; j < P; j++) {
+            before += R.ids[j] < e;
+            at += R.ids[j] == e;
+        }
+        p.offsets[e] = before;
+        if (p.dbg_offsets) p.dbg_offsets[e] = before;
         if (e < p.E) {
-            const int c = __popc(emask[e]);
-            p.counts[e] = c;
-            if (p.dbg_counts) p.dbg_counts[e] = c;
+            p.counts[e] = at;
+            if (p.dbg_counts) p.dbg_counts[e] = at;
         }
     }
     if (threadIdx.x == 0) p.cnt[kCntUniq] = R.U;
@@ -183,13 +205,33 @@ struct ItemRef {
     bool valid;
 };
 
+// A run of at most kMaxRoundsPerWarp consecutive K rounds of one item.
+struct Chunk {
+    int item, r0, r1;   // r1 == 0: none
+};
+
+// Next chunk of the unit range [x, end) (units = item * R + round); advances x.
+__device__ inline Chunk take_chunk(int &x, int end, int R) {
+    Chunk c{0, 0, 0};
+    if (x < end) {
+        c.item = x / R;
+        c.r0 = x - c.item * R;
+        c.r1 = min(min(R, c.r0 + kMaxRoundsPerWarp), end - c.item * R);
+        x = c.item * R + c.r1;
+    }
+    return c;
+}
+
+// MODE 0 item = (used expert u, 8 intermediates): A rows g are gate rows, rows
+// g+8 the up rows of the same intermediate index. MODE 1 item = (u, 16 hidden
+// rows).
 template <int MODE>
-__device__ inline ItemRef item_ref(const Params &p, const DecRoute &R, int item, int items) {
-    ItemRef r{0, 0, 0, item < items};
+__device__ inline ItemRef item_of(const Params &p, const DecRoute &R, const Chunk &c) {
+    ItemRef r{0, 0, 0, c.r1 > 0};
     if (r.valid) {
         const int per_u = MODE == 0 ? p.I / 8 : p.H / 16;
-        r.u = item / per_u;
-        r.m0 = (item % per_u) * (MODE == 0 ? 8 : 16);
+        r.u = c.item / per_u;
+        r.m0 = (c.item - r.u * per_u) * (MODE == 0 ? 8 : 16);
         r.e = R.uniq[r.u];
     }
     return r;
@@ -226,44 +268,6 @@ __device__ inline void issue_loads(const Params &p, const ItemRef &it, int g, in
     }
 }
 
-// Grid-wide barrier for a cooperatively launched grid (all CTAs co-resident),
-// used once per kernel. Each CTA reads the generation word, then arrives on the
-// count; the last to arrive advances the generation (which the others poll) and
-// only then resets the count, so the release costs two dependent atomics and the
-// words (in the handle's device status block) are ready for the next launch. The
-// wait is bounded: after `limit_ns` it latches NVFP4_MOE_ERR_TIMEOUT and returns.
-__device__ inline void grid_barrier_once(int32_t *status, uint64_t limit_ns = 200000000ull) {
-    unsigned *gen = reinterpret_cast<unsigned *>(status + kStatusBarGen);
-    unsigned *count = reinterpret_cast<unsigned *>(status + kStatusBarTop);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        volatile unsigned *vgen = gen;
-        const unsigned my_gen = *vgen;
-        __threadfence();
-        if (atomicAdd(count, 1u) + 1u == gridDim.x) {
-            atomicAdd(gen, 1u);
-            atomicExch(count, 0u);
-        } else {
-            const uint64_t t0 = globaltimer();
-            while (*vgen == my_gen) {
-                __nanosleep(20);
-                if (globaltimer() - t0 > limit_ns) {
-                    latch_status(status, NVFP4_MOE_ERR_TIMEOUT, 100);
-                    break;
-                }
-            }
-        }
-        __threadfence();
-    }
-    __syncthreads();
-}
-
-struct DecSmem {
-    float *red;     // [8 warps][32][4] split-K partial sums
-    __half *xs;     // [8 token slots][H+4] F16 activations
-    uint8_t *raw;   // [T][H] raw BF16 / int8 activations (cp.async at kernel start)
-};
-
 __device__ inline void cp_async16(void *smem, const void *gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
                  : "memory");
@@ -296,147 +300,181 @@ __device__ inline void act8(const Params &p, const uint8_t *raw, int t, int k8, 
     }
 }
 
-// The weight-streaming passes of one projection over this CTA's share of the
-// items. MODE 0: gate/up + SwiGLU; item = (unique expert u, 8 intermediate rows):
-// A rows g are gate rows, rows g+8 the up rows of the same intermediate index,
-// so each thread ends with g and u of the same (row, token) pair. MODE 1: down +
-// weighted combine; item = (unique expert u, 16 hidden rows); B = h of the pairs
-// (token, u), zero for tokens not routed to u. Each pass covers kDecWarps/split
-// items; the next pass's loads are issued before the current pass computes (two
-// register buffers). On entry buf0 already holds this CTA's first pass.
-template <int MODE>
-__device__ inline void run_passes(const Params &p, const DecRoute &R, const DecSmem &S,
-                                  PassBuf &buf0, PassBuf &buf1) {
-    const int H = p.H, I = p.I, T = p.T;
-    const int rounds = (MODE == 0 ? H : I) / 128;
-    const int split = k_split(rounds);
-    const int rpw = cdiv(rounds, split);
-    const int ipc = kDecWarps / split;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int items = R.U * ((MODE == 0 ? I : H) / (MODE == 0 ? 8 : 16));
-    const int item_l = warp / split, part = warp % split;
-    const int r_begin = part * rpw, r_end = min(rounds, r_begin + rpw);
-    const int stride = gridDim.x * ipc;
-    const int ld = H + 4;
-    const __half *xrow = S.xs + g * ld + 32 * q;
-    int base = blockIdx.x * ipc;
-    ItemRef cur = item_ref<MODE>(p, R, base + item_l, items);
 
-    auto pass_step = [&](PassBuf &b, PassBuf &nb) {
-        const ItemRef nxt = item_ref<MODE>(p, R, base + stride + item_l, items);
-        issue_loads<MODE>(p, nxt, g, q, r_begin, r_end, nb);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (cur.valid) {
-            const int mypos = (MODE == 1 && g < T) ? R.upos[cur.u * kSlots + g] : -1;
-            const __half *hrow = p.h + (size_t)(mypos < 0 ? 0 : mypos) * I + 32 * q;
+// Bounded wait until *word >= target (one thread); latches TIMEOUT on give-up.
+__device__ inline bool wait_geq(const int32_t *word, int target, int32_t *status, int where) {
+    const volatile int32_t *v = word;
+    if (*v >= target) return true;
+    const uint64_t t0 = globaltimer();
+    while (*v < target) {
+        __nanosleep(64);
+        if (globaltimer() - t0 > kDecWaitNs) {
+            latch_status(status, NVFP4_MOE_ERR_TIMEOUT, where);
+            return false;
+        }
+    }
+    return true;
+}
+
+struct DecSmem {
+    __half *xs;     // [8 token slots][H+4] F16 activations
+    uint8_t *raw;   // [T][H] raw BF16 / int8 activations (cp.async at kernel start)
+    __half *hs;     // [hs_rows][I+8] h rows of this CTA's phase-2 experts
+};
+
+// Phase 1 end of an item segment (nr rounds of the item's R1 done here).
+__device__ inline void flush_gateup(const Params &p, const DecRoute &R, const ItemRef &it, int nr,
+                                    int R1, const float (&acc)[4], int g, int q, int lane) {
+    const int I = p.I;
+    const int item = it.u * (I / 8) + it.m0 / 8;
+    int32_t *ds = p.dstate;
+    float *gu = p.dgu;
+    bool finisher = true;
+    if (nr != R1) {
 #pragma unroll
-            for (int j = 0; j < kMaxRoundsPerWarp; j++) {
-                const int r = r_begin + j;
-                if (r < r_end) {
-                    if (MODE == 0) {
-                        const __half *xr = xrow + 128 * r;
-                        round_mma(acc, b.ca[j], b.cb[j], b.sa[j], b.sb[j],
-                                  [&](int s, uint32_t &x0, uint32_t &x1) {
-                                      const uint2 v = *reinterpret_cast<const uint2 *>(xr + 4 * s);
-                                      x0 = v.x;
-                                      x1 = v.y;
-                                  });
-                    } else {
-                        uint4 hv[4];
-#pragma unroll
-                        for (int v = 0; v < 4; v++)
-                            hv[v] = mypos >= 0 ? reinterpret_cast<const uint4 *>(hrow + 128 * r)[v]
-                                               : make_uint4(0, 0, 0, 0);
-                        round_mma(acc, b.ca[j], b.cb[j], b.sa[j], b.sb[j],
-                                  [&](int s, uint32_t &x0, uint32_t &x1) {
-                                      const uint4 &w = hv[s >> 1];
-                                      x0 = (s & 1) ? w.z : w.x;
-                                      x1 = (s & 1) ? w.w : w.y;
-                                  });
-                    }
-                }
+        for (int c = 0; c < 2; c++) {
+            const int tok = 2 * q + c;
+            const int pos = tok < p.T ? R.upos[it.u * kSlots + tok] : -1;
+            if (pos >= 0) {
+                atomicAdd(gu + ((size_t)2 * pos) * I + it.m0 + g, acc[c]);
+                atomicAdd(gu + ((size_t)2 * pos + 1) * I + it.m0 + g, acc[2 + c]);
             }
         }
-        if (split > 1) {
-            *reinterpret_cast<float4 *>(S.red + (warp * 32 + lane) * 4) =
-                make_float4(acc[0], acc[1], acc[2], acc[3]);
-            __syncthreads();
-            if (part == 0) {
-                for (int w2 = 1; w2 < split; w2++) {
-                    const float4 o = *reinterpret_cast<const float4 *>(S.red + ((warp + w2) * 32 + lane) * 4);
-                    acc[0] += o.x;
-                    acc[1] += o.y;
-                    acc[2] += o.z;
-                    acc[3] += o.w;
-                }
-            }
-            __syncthreads();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+            __threadfence();
+            last = atomicAdd(ds + kDsItems + item, nr) + nr == R1;
         }
-        if (part == 0 && cur.valid) {
-            if (MODE == 0) {
-                const float sgl = p.gate_global[cur.e], sul = p.up_global[cur.e];
+        finisher = __shfl_sync(0xffffffffu, last, 0) != 0;
+        if (!finisher) return;
+        __threadfence();
+    }
+    const float sg = p.gate_global[it.e], su = p.up_global[it.e];
 #pragma unroll
-                for (int c = 0; c < 2; c++) {
-                    const int tok = 2 * q + c;
-                    const int pos = tok < T ? R.upos[cur.u * kSlots + tok] : -1;
-                    if (pos >= 0) {
-                        const float gv = acc[c] * sgl * R.xsc[tok], uv = acc[2 + c] * sul * R.xsc[tok];
-                        p.h[(size_t)pos * I + cur.m0 + g] = __float2half_rn(silu(gv) * uv);
-                    }
-                }
-            } else {
-                const float sd = p.down_global[cur.e];
-#pragma unroll
-                for (int c = 0; c < 2; c++) {
-                    const int tok = 2 * q + c;
-                    if (tok < T && R.upos[cur.u * kSlots + tok] >= 0) {
-                        const float w = R.uw[cur.u * kSlots + tok] * sd;
-                        atomicAdd(p.out + (size_t)tok * H + cur.m0 + g, acc[c] * w);
-                        atomicAdd(p.out + (size_t)tok * H + cur.m0 + g + 8, acc[2 + c] * w);
-                    }
-                }
+    for (int c = 0; c < 2; c++) {
+        const int tok = 2 * q + c;
+        const int pos = tok < p.T ? R.upos[it.u * kSlots + tok] : -1;
+        if (pos >= 0) {
+            float gs = acc[c], us = acc[2 + c];
+            if (nr != R1) {   // the item's full sums; leaves the accumulator cleared
+                gs = atomicExch(gu + ((size_t)2 * pos) * I + it.m0 + g, 0.0f);
+                us = atomicExch(gu + ((size_t)2 * pos + 1) * I + it.m0 + g, 0.0f);
             }
+            const float gv = gs * sg * R.xsc[tok], uv = us * su * R.xsc[tok];
+            p.h[(size_t)pos * I + it.m0 + g] = __float2half_rn(silu(gv) * uv);
         }
-        cur = nxt;
-        base += stride;
-    };
-    while (base < items) {
-        pass_step(buf0, buf1);
-        if (base >= items) break;
-        pass_step(buf1, buf0);
+    }
+    __syncwarp();
+    if (lane == 0) {
+        if (nr != R1) atomicExch(ds + kDsItems + item, 0);
+        __threadfence();
+        atomicAdd(ds + kDsReady + it.u, 1);
     }
 }
 
-template <int MODE>
-__device__ inline void first_loads(const Params &p, const DecRoute &R, PassBuf &b) {
-    const int rounds = (MODE == 0 ? p.H : p.I) / 128;
-    const int split = k_split(rounds);
-    const int rpw = cdiv(rounds, split);
-    const int ipc = kDecWarps / split;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int items = R.U * ((MODE == 0 ? p.I : p.H) / (MODE == 0 ? 8 : 16));
-    const int part = warp % split, r_begin = part * rpw;
-    const ItemRef it = item_ref<MODE>(p, R, blockIdx.x * ipc + warp / split, items);
-    issue_loads<MODE>(p, it, lane >> 2, lane & 3, r_begin, min(rounds, r_begin + rpw), b);
+// Phase 2 end of an item segment: the weighted partial sums into out.
+__device__ inline void flush_down(const Params &p, const DecRoute &R, const ItemRef &it,
+                                  const float (&acc)[4], int g, int q) {
+    const float sd = p.down_global[it.e];
+#pragma unroll
+    for (int c = 0; c < 2; c++) {
+        const int tok = 2 * q + c;
+        if (tok < p.T && R.upos[it.u * kSlots + tok] >= 0) {
+            const float w = R.uw[it.u * kSlots + tok] * sd;
+            atomicAdd(p.out + (size_t)tok * p.H + it.m0 + g, acc[c] * w);
+            atomicAdd(p.out + (size_t)tok * p.H + it.m0 + g + 8, acc[2 + c] * w);
+        }
+    }
 }
 
-// The whole decode layer in one cooperatively launched grid: every CTA routes
-// the <= 8 tokens itself, stages the F16 activations, streams its share of the
-// gate/up weights (SwiGLU into h), issues its first down-projection loads, and
-// after one grid-wide barrier (h complete, out cleared) streams its share of the
-// down weights with the weighted combine.
+// Streams the warp's unit range [x, end) of one projection; `cur` (already in
+// buf0) is its first chunk. Loads of the next chunk are issued before the current
+// chunk computes (two register buffers).
+template <int MODE>
+__device__ inline void run_range(const Params &p, const DecRoute &R, const DecSmem &S, int &x,
+                                 int end, Chunk cur, PassBuf &buf0, PassBuf &buf1, int hs_pos0) {
+    const int H = p.H, I = p.I, T = p.T;
+    const int RR = (MODE == 0 ? H : I) / 128;
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int ld = H + 4, ldh = I + 8;
+    const __half *xrow = S.xs + g * ld + 32 * q;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int seg_r0 = cur.r0;
+
+    auto step = [&](PassBuf &b, PassBuf &nb) {
+        const Chunk nxt = take_chunk(x, end, RR);
+        issue_loads<MODE>(p, item_of<MODE>(p, R, nxt), g, q, nxt.r0, nxt.r1, nb);
+        const ItemRef it = item_of<MODE>(p, R, cur);
+        const int mypos = (MODE == 1 && g < T) ? R.upos[it.u * kSlots + g] : -1;
+        const __half *hrow = S.hs + (size_t)(mypos < 0 ? 0 : mypos - hs_pos0) * ldh + 32 * q;
+#pragma unroll
+        for (int j = 0; j < kMaxRoundsPerWarp; j++) {
+            const int r = cur.r0 + j;
+            if (r < cur.r1) {
+                if (MODE == 0) {
+                    const __half *xr = xrow + 128 * r;
+                    round_mma(acc, b.ca[j], b.cb[j], b.sa[j], b.sb[j],
+                              [&](int s, uint32_t &x0, uint32_t &x1) {
+                                  const uint2 v = *reinterpret_cast<const uint2 *>(xr + 4 * s);
+                                  x0 = v.x;
+                                  x1 = v.y;
+                              });
+                } else {
+                    uint4 hv[4];
+#pragma unroll
+                    for (int v = 0; v < 4; v++)
+                        hv[v] = mypos >= 0 ? reinterpret_cast<const uint4 *>(hrow + 128 * r)[v]
+                                           : make_uint4(0, 0, 0, 0);
+                    round_mma(acc, b.ca[j], b.cb[j], b.sa[j], b.sb[j],
+                              [&](int s, uint32_t &x0, uint32_t &x1) {
+                                  const uint4 &w = hv[s >> 1];
+                                  x0 = (s & 1) ? w.z : w.x;
+                                  x1 = (s & 1) ? w.w : w.y;
+                              });
+                }
+            }
+        }
+        if (nxt.r1 == 0 || nxt.item != cur.item) {
+            if (MODE == 0)
+                flush_gateup(p, R, it, cur.r1 - seg_r0, RR, acc, g, q, lane);
+            else
+                flush_down(p, R, it, acc, g, q);
+#pragma unroll
+            for (int c = 0; c < 4; c++) acc[c] = 0.0f;
+            seg_r0 = nxt.r0;
+        }
+        cur = nxt;
+    };
+    while (cur.r1 > 0) {
+        step(buf0, buf1);
+        if (cur.r1 == 0) break;
+        step(buf1, buf0);
+    }
+}
+
+// [a, b) = this warp's share of n units when the grid's W workers split them
+// evenly in contiguous ranges.
+__device__ inline void share(int n, int w, int W, int &a, int &b) {
+    a = (int)((long long)n * w / W);
+    b = (int)((long long)n * (w + 1) / W);
+}
+
 template <int NPER>
-__global__ void __launch_bounds__(kDecThreads, 2) decode_layer_kernel(Params p) {
+__global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) {
     extern __shared__ __align__(16) uint8_t dsm[];
     __shared__ DecRoute R;
-    const int H = p.H, T = p.T;
-    DecSmem S;
-    S.red = reinterpret_cast<float *>(dsm);
-    int *emask = reinterpret_cast<int *>(dsm + kDecWarps * 32 * 4 * sizeof(float));
-    int *cnt = emask + p.E;
-    S.xs = reinterpret_cast<__half *>(cnt + p.E);
-    S.raw = reinterpret_cast<uint8_t *>(S.xs + kSlots * (H + 4));
+    const int H = p.H, I = p.I, T = p.T;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ld = H + 4;
+    DecSmem S;
+    S.xs = reinterpret_cast<__half *>(dsm);
+    S.raw = reinterpret_cast<uint8_t *>(S.xs + kSlots * ld);
+    S.hs = reinterpret_cast<__half *>(S.raw + T * raw_act_bytes(p.act_type, H));
+    int32_t *ds = p.dstate;
+
+    // Everything this layer reads may come from the previous kernel in the stream.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // the activations first: their loads are then not queued behind the weights'
     const int raw_bytes = T * raw_act_bytes(p.act_type, H);
@@ -444,12 +482,21 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_layer_kernel(Params p) 
         cp_async16(S.raw + 16 * c, static_cast<const uint8_t *>(p.act) + 16 * c);
     asm volatile("cp.async.commit_group;" ::: "memory");
 
-    cta_route<NPER>(p, R, emask, cnt, blockIdx.x == 0);
+    cta_route<NPER>(p, R, blockIdx.x == 0);
+    const int U = R.U;
+
+    // phase-1 share of this warp and its first loads
+    const int R1 = H / 128, R2 = I / 128;
+    const int n1 = U * (I / 8) * R1, n2 = U * (H / 16) * R2;
+    int a1, b1;
+    share(n1, blockIdx.x * kDecWarps + warp, gridDim.x * kDecWarps, a1, b1);
+    int x1 = a1;
+    const Chunk c1 = take_chunk(x1, b1, R1);
     PassBuf buf0, buf1;
-    first_loads<0>(p, R, buf0);
+    issue_loads<0>(p, item_of<0>(p, R, c1), lane >> 2, lane & 3, c1.r0, c1.r1, buf0);
 
     // per-token amax -> power-of-two shift -> F16 activations in shared memory
-    // (token slots past T are zeros); every load of x is issued before its use
+    // (token slots past T are zeros)
     const int n8 = H / 8;
     for (int c = threadIdx.x; c < (kSlots - T) * n8; c += blockDim.x) {
         uint2 *dst = reinterpret_cast<uint2 *>(S.xs + (T + c / n8) * ld + 8 * (c % n8));
@@ -459,9 +506,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_layer_kernel(Params p) 
     if (threadIdx.x < kSlots) R.amax[threadIdx.x] = 0u;
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    // two passes over the shared raw copy (global memory for FP32 input): the
-    // per-token amax (reduced per warp, one shared atomic per warp and token),
-    // then the shifted F16 values. Loop bounds are whole warps for the shuffles.
     const int ngrp = T * n8, ngrp_w = (ngrp + 31) & ~31;
     if (p.act_type != NVFP4_MOE_ACT_INT8) {
         for (int c = threadIdx.x; c < ngrp_w; c += blockDim.x) {
@@ -479,7 +523,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_layer_kernel(Params p) 
             const unsigned mb = __float_as_uint(m);
             const unsigned m_lo = __reduce_max_sync(0xffffffffu, t == lo_t ? mb : 0u);
             const unsigned m_hi = __reduce_max_sync(0xffffffffu, t != lo_t ? mb : 0u);
-            if ((threadIdx.x & 31) == 0) {
+            if (lane == 0) {
                 if (lo_t < (unsigned)T) atomicMax(&R.amax[lo_t], m_lo);
                 if (hi_t != lo_t && hi_t < (unsigned)T) atomicMax(&R.amax[hi_t], m_hi);
             }
@@ -500,18 +544,70 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_layer_kernel(Params p) 
         R.xsc[threadIdx.x] = p.act_type == NVFP4_MOE_ACT_INT8
                                  ? p.act_scale[threadIdx.x]
                                  : exp2i(-pow2_shift_for(__uint_as_float(R.amax[threadIdx.x])));
-    if (blockIdx.x == 0) publish_route(p, R, emask, cnt);
-    // out is cleared for the combine before the grid barrier below; act never
-    // aliases out in this mode (only an accumulating call may pass act == out)
-    if (!p.out_add)
-        for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < T * H / 4; c += gridDim.x * blockDim.x)
+    if (blockIdx.x == 0) publish_route(p, R);
+    // this CTA's stripe of out is cleared for the combine (unless accumulating)
+    if (!p.out_add) {
+        int za, zb;
+        share(T * H / 4, blockIdx.x, gridDim.x, za, zb);
+        for (int c = za + threadIdx.x; c < zb; c += blockDim.x)
             reinterpret_cast<float4 *>(p.out)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     __syncthreads();
+    // the activations are read and this stripe of out is cleared: phase-2 adds
+    // anywhere into out wait for every CTA to get here (out may alias act)
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ds + kDsStaged, 1);
+    }
 
-    run_passes<0>(p, R, S, buf0, buf1);
-    first_loads<1>(p, R, buf0);     // down weights in flight while the grid catches up
-    grid_barrier_once(p.status);    // h complete, out cleared
-    run_passes<1>(p, R, S, buf0, buf1);
+    run_range<0>(p, R, S, x1, b1, c1, buf0, buf1, 0);
+
+    // phase 2: this CTA's share, split evenly over its warps
+    int ca, cb;
+    share(n2, blockIdx.x, gridDim.x, ca, cb);
+    int a2, b2;
+    share(cb - ca, warp, kDecWarps, a2, b2);
+    a2 += ca;
+    b2 += ca;
+    int x2 = a2;
+    const Chunk c2 = take_chunk(x2, b2, R2);
+    issue_loads<1>(p, item_of<1>(p, R, c2), lane >> 2, lane & 3, c2.r0, c2.r1, buf0);
+    const int per_u2 = (H / 16) * R2;
+    const int u_lo = ca / per_u2, u_hi = cb > ca ? (cb - 1) / per_u2 : u_lo - 1;
+    const int pos_lo = u_hi >= u_lo ? R.uoff[u_lo] : 0;
+    const int rows = u_hi >= u_lo ? R.uoff[u_hi + 1] - pos_lo : 0;
+    __syncthreads();
+    if (threadIdx.x == 0 && u_hi >= u_lo) {
+        bool ok = wait_geq(ds + kDsStaged, gridDim.x, p.status, 101);
+        for (int u = u_lo; ok && u <= u_hi; u++) ok = wait_geq(ds + kDsReady + u, I / 8, p.status, 102);
+        if (rows > p.dec_hs_rows) latch_status(p.status, NVFP4_MOE_ERR_UNSUPPORTED_DIMS, 103);
+        __threadfence();
+    }
+    __syncthreads();
+    {
+        const int nrow = min(rows, p.dec_hs_rows), per_row = I / 8;   // 16-byte pieces per h row
+        for (int c = threadIdx.x; c < nrow * per_row; c += blockDim.x) {
+            const int r = c / per_row, k = c - r * per_row;
+            cp_async16(S.hs + (size_t)r * (I + 8) + 8 * k, p.h + (size_t)(pos_lo + r) * I + 8 * k);
+        }
+        asm volatile("cp.async.commit_group;\n cp.async.wait_all;" ::: "memory");
+    }
+    __syncthreads();
+    if (rows <= p.dec_hs_rows) run_range<1>(p, R, S, x2, b2, c2, buf0, buf1, pos_lo);
+
+    // The next layer's grid may launch once every CTA is here; the last CTA to
+    // finish resets the counts for the next launch.
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(ds + kDsExit, 1) == (int)gridDim.x - 1) {
+            for (int u = 0; u < U; u++) ds[kDsReady + u] = 0;
+            ds[kDsStaged] = 0;
+            __threadfence();
+            ds[kDsExit] = 0;
+        }
+    }
+    asm volatile("griddepcontrol.launch_dependents;" :::);
 }
 
 static int sm_count() {
@@ -521,27 +617,35 @@ static int sm_count() {
     return sms;
 }
 
+// h rows one CTA's phase-2 range can touch: a range of at most
+// ceil(U * per_u / G) units touches at most floor(U / G) + 2 used experts, each
+// with at most T pairs.
+int decode_hs_rows(int T, int K, int E, int grid) {
+    const int P = T * K, U_max = P < E ? P : E;
+    const int r = (U_max / grid + 2) * T;
+    return r < P ? r : P;
+}
+
+int decode_grid() { return sm_count(); }
+
 static size_t decode_smem(const Params &p) {
-    return kDecWarps * 32 * 4 * sizeof(float) + 2 * (size_t)p.E * sizeof(int) +
-           (size_t)8 * (p.H + 4) * sizeof(__half) + (size_t)p.T * raw_act_bytes(p.act_type, p.H);
+    return (size_t)kSlots * (p.H + 4) * sizeof(__half) + (size_t)p.T * raw_act_bytes(p.act_type, p.H) +
+           (size_t)p.dec_hs_rows * (p.I + 8) * sizeof(__half);
 }
 
 template <int NPER>
 static cudaError_t launch_layer(const Params &p, cudaStream_t s) {
-    const size_t smem = decode_smem(p);
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_layer_kernel<NPER>,
-                                                                  kDecThreads, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    const int U_max = min(p.T * p.K, p.E);
-    const int need = max(cdiv(U_max * (p.I / 8), kDecWarps / k_split(p.H / 128)),
-                         cdiv(U_max * (p.H / 16), kDecWarps / k_split(p.I / 128)));
-    const int grid = max(1, min(min(per_sm, 2) * sm_count(), need));
-    Params pp = p;
-    void *args[] = {&pp};
-    return cudaLaunchCooperativeKernel((const void *)decode_layer_kernel<NPER>, dim3(grid),
-                                       dim3(kDecThreads), args, smem, s);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(decode_grid());
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = decode_smem(p);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_layer_kernel<NPER>, p);
 }
 
 cudaError_t launch_decode(const Params &p, cudaStream_t s) {

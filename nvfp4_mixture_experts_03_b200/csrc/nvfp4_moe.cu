@@ -26,6 +26,9 @@ struct nvfp4_moe {
     int pf_clusters;  // resident CTA pairs of the prefill GEMMs
     CodeMaps codes;   // tensor maps of the weight code planes (prefill GEMMs)
     int32_t *status;  // kStatusWords ints on the device
+    uint8_t *dstate;  // decode state (zero between launches), for dec_pairs pairs
+    size_t dstate_bytes;
+    int dec_pairs;
     cudaEvent_t phase[NVFP4_MOE_PHASE_EVENTS];
     bool phase_on;
 };
@@ -197,10 +200,18 @@ int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
         return NVFP4_MOE_ERR_CUDA;
     }
     h->status = nullptr;
+    h->dstate = nullptr;
     h->phase_on = false;
+    const int dec_t = d.max_tokens < NVFP4_MOE_DECODE_MAX_T ? d.max_tokens : NVFP4_MOE_DECODE_MAX_T;
+    h->dec_pairs = dec_t * d.top_k;
+    h->dstate_bytes = h->dec_pairs > 0 ? decode_state_bytes(h->dec_pairs, d.inter) : 0;
     if (cudaMalloc(&h->status, kStatusWords * sizeof(int32_t)) != cudaSuccess ||
-        cudaMemset(h->status, 0, kStatusWords * sizeof(int32_t)) != cudaSuccess) {
+        cudaMemset(h->status, 0, kStatusWords * sizeof(int32_t)) != cudaSuccess ||
+        (h->dstate_bytes &&
+         (cudaMalloc(&h->dstate, h->dstate_bytes) != cudaSuccess ||
+          cudaMemset(h->dstate, 0, h->dstate_bytes) != cudaSuccess))) {
         if (h->status) cudaFree(h->status);
+        if (h->dstate) cudaFree(h->dstate);
         delete h;
         return NVFP4_MOE_ERR_CUDA;
     }
@@ -289,6 +300,12 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     p.nch = L.nch;
     p.max_tiles_gu = L.max_gu;
     p.max_tiles_dn = L.max_dn;
+    if (T <= NVFP4_MOE_DECODE_MAX_T) {
+        if (T * d.top_k > h->dec_pairs || !h->dstate) return NVFP4_MOE_ERR_INVALID_ARG;
+        p.dstate = reinterpret_cast<int32_t *>(h->dstate);
+        p.dgu = reinterpret_cast<float *>(h->dstate + decode_state_ints_bytes(h->dec_pairs, d.inter));
+        p.dec_hs_rows = decode_hs_rows(T, d.top_k, d.n_experts, decode_grid());
+    }
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // External records, so that a forward captured into a CUDA graph records the
@@ -341,6 +358,9 @@ int nvfp4_moe_get_status(nvfp4_moe_t *h, void *stream) {
     if (cudaMemcpy(st, h->status, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
         return NVFP4_MOE_ERR_CUDA;
     if (cudaMemset(h->status, 0, sizeof(st)) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
+    // A launch that gave up may have left decode counts or partial sums behind.
+    if (st[kStatusCode] != 0 && h->dstate && cudaMemset(h->dstate, 0, h->dstate_bytes) != cudaSuccess)
+        return NVFP4_MOE_ERR_CUDA;
     return st[kStatusCode];
 }
 
@@ -361,6 +381,7 @@ int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events, int32_t n_ev
 void nvfp4_moe_destroy(nvfp4_moe_t *h) {
     if (!h) return;
     if (h->status) cudaFree(h->status);
+    if (h->dstate) cudaFree(h->dstate);
     delete h;
 }
 
@@ -378,8 +399,8 @@ void nvfp4_moe_destroy(nvfp4_moe_t *h) {
 // library holds until the process exits.
 namespace {
 
-constexpr size_t kStaticScratchBytes = size_t(1) << 20;  // 1 MiB per device
-constexpr size_t kStaticStatusBytes = 256;               // status words, then the workspace
+constexpr size_t kStaticScratchBytes = size_t(2) << 20;  // 2 MiB per device
+constexpr size_t kStaticStatusBytes = 256;               // status words, then decode state, workspace
 constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
@@ -437,8 +458,10 @@ int nvfp4_moe_forward_decode_static(const nvfp4_moe_dims *dims, const nvfp4_moe_
     if (io->T < 0 || io->T > dims->max_tokens) return NVFP4_MOE_ERR_INVALID_ARG;
     if (io->T > NVFP4_MOE_DECODE_MAX_T) return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
     if (io->T == 0) return NVFP4_MOE_OK;
+    const int pairs = io->T * dims->top_k;
+    const size_t state = decode_state_bytes(pairs, dims->inter);
     const size_t need = layout(*dims, io->T).total;
-    if (need > kStaticScratchBytes - kStaticStatusBytes) return NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (need + state > kStaticScratchBytes - kStaticStatusBytes) return NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_MOE_ERR_NO_DEVICE;
     int major = 0, sms = 0;
@@ -457,12 +480,17 @@ int nvfp4_moe_forward_decode_static(const nvfp4_moe_dims *dims, const nvfp4_moe_
     h.num_sms = sms;
     h.pf_clusters = 0;   // T <= 8 never reaches the prefill GEMMs
     h.status = reinterpret_cast<int32_t *>(scratch);
+    h.dstate = scratch + kStaticStatusBytes;
+    h.dstate_bytes = state;
+    h.dec_pairs = pairs;
     h.phase_on = false;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // The status words must start at zero (they latch the first device error).
-    if (cudaMemsetAsync(scratch, 0, kStaticStatusBytes, s) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
-    return nvfp4_moe_forward(&h, io, scratch + kStaticStatusBytes,
-                             kStaticScratchBytes - kStaticStatusBytes, stream);
+    // The status words and the decode state must start at zero (the status
+    // latches the first device error; an earlier call that gave up may have left
+    // decode counts behind, and no status read follows a call here).
+    if (cudaMemsetAsync(scratch, 0, kStaticStatusBytes + state, s) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
+    return nvfp4_moe_forward(&h, io, scratch + kStaticStatusBytes + state,
+                             kStaticScratchBytes - kStaticStatusBytes - state, stream);
 }
 
 }  // extern "C"

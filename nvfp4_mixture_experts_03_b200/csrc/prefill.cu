@@ -55,6 +55,7 @@ constexpr int kRawStages = 4;                  // 16 K steps of weights in fligh
 constexpr int kRawCodeBytes = kBM * kRawSteps * 32;   // 128 rows x 128 B of E2M1 codes
 constexpr int kRawScaleBytes = kBM * kRawSteps * 4;   // 128 rows x 16 B of E4M3 scales
 constexpr int kRawBytes = kRawCodeBytes + kRawScaleBytes;
+static_assert(kRing % 2 == 0 && kRawSteps % 2 == 0, "the dequant warps fill ring stages in pairs");
 constexpr int kTmemCols = 512;                 // two 256-column accumulators
 constexpr int kEpiBytes = 2 * 32 * kBM * 2;    // epilogue staging: 2 x (32 columns x 128 rows x F16)
 constexpr int kColBytes = kBN * 4;            // the tile's per-column factors (FP32)
@@ -234,9 +235,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         Ring<kRawStages> rr;
         uint4 s4 = make_uint4(0, 0, 0, 0);
         bool ok = true;
+        // Two K steps (two ring stages) per iteration: K is a multiple of 128, so
+        // every tile has an even number of steps and the pair never wraps the ring
+        // (kRing is even); one proxy fence and one pass of waits per pair.
         for (int tl = 0; ok && tl < ntl; tl++) {
-            for (int kk = 0; kk < nk; kk++) {
-                const int kq = kk % kRawSteps;
+            for (int kk = 0; kk < nk; kk += 2) {
+                const int kq = kk % kRawSteps;   // 0 or 2
                 const uint8_t *raw = raw_base + rr.stage * kRawBytes;
                 if (kq == 0) {
                     const bool g = mbar_wait(&bars->raw_full[rr.stage], rr.phase, abort, p.status, 9);
@@ -246,20 +250,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     s4 = *reinterpret_cast<const uint4 *>(raw + scale_off);
                 }
-                const bool got = mbar_wait(&bars->empty[ring.stage], ring.phase ^ 1, abort, p.status, 1);
+                const int s0 = ring.stage, s1 = ring.stage + 1;
+                const bool got = mbar_wait(&bars->empty[s0], ring.phase ^ 1, abort, p.status, 1) &&
+                                 mbar_wait(&bars->empty[s1], ring.phase ^ 1, abort, p.status, 1);
                 if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
                     break;
                 }
-                const int c = 2 * kq + hf;
-                const uint4 code = *reinterpret_cast<const uint4 *>(raw + code_off + ((c ^ swz) << 4));
-                const uint32_t sw = kq == 0 ? s4.x : kq == 1 ? s4.y : kq == 2 ? s4.z : s4.w;
-                store_half_row(a_base + ring.stage * kAStage, r, hf, code, sw >> (16 * hf));
+                const uint4 code0 = *reinterpret_cast<const uint4 *>(raw + code_off + (((2 * kq + hf) ^ swz) << 4));
+                const uint4 code1 = *reinterpret_cast<const uint4 *>(raw + code_off + (((2 * kq + 2 + hf) ^ swz) << 4));
+                const uint32_t sw0 = kq == 0 ? s4.x : s4.z, sw1 = kq == 0 ? s4.y : s4.w;
+                store_half_row(a_base + s0 * kAStage, r, hf, code0, sw0 >> (16 * hf));
+                store_half_row(a_base + s1 * kAStage, r, hf, code1, sw1 >> (16 * hf));
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(mapa_shared(&bars->a_full[ring.stage], 0));
+                if (lane == 0) {
+                    mbar_arrive_cluster(mapa_shared(&bars->a_full[s0], 0));
+                    mbar_arrive_cluster(mapa_shared(&bars->a_full[s1], 0));
+                }
                 ring.next();
-                if (kq == kRawSteps - 1 || kk == nk - 1) {
+                ring.next();
+                if (kq + 1 == kRawSteps - 1 || kk + 2 == nk) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->raw_empty[rr.stage]);
                     rr.next();
