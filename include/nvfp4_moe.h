@@ -43,14 +43,24 @@
  *   - Every pointer in nvfp4_moe_weights and nvfp4_moe_io is a DEVICE pointer
  *     owned by the caller. The handle BORROWS the weight pointers: they must stay
  *     valid until nvfp4_moe_destroy. The library allocates no device memory
- *     except one 256-byte status block made by nvfp4_moe_create.
- *   - All scratch lives in the caller's workspace (nvfp4_moe_workspace_bytes).
+ *     except what nvfp4_moe_create makes: a 256-byte status block and, when
+ *     max_tokens >= 1, the decode state (a few counters plus FP32 partial sums
+ *     of min(max_tokens, 8) * top_k token slots x 2 x inter: 0.5 MB for the
+ *     512-expert, 2048/768, top-10 layer), kept zero between calls.
+ *   - All other scratch lives in the caller's workspace (nvfp4_moe_workspace_bytes).
  *
  * Errors: every call returns 0 (NVFP4_MOE_OK) or a negative nvfp4_moe_status.
  *   Host-side checks run before anything is enqueued; a call that fails them
  *   enqueues nothing. Conditions found on the device (routing id out of range
- *   or duplicated, a non-finite routing logit) are latched in the status block
- *   and returned by nvfp4_moe_get_status. forward never synchronises.
+ *   or duplicated, a non-finite routing logit, a wait that gave up) are latched
+ *   in the status block and returned by nvfp4_moe_get_status. forward never
+ *   synchronises. Every device-side wait is bounded: a kernel whose wait runs
+ *   out latches NVFP4_MOE_ERR_TIMEOUT and returns instead of hanging.
+ *
+ * Co-residency: the decode kernel (T <= 8) runs one CTA per SM and its CTAs wait
+ *   on one another through counters (bounded). It assumes the GPU is not shared
+ *   with other work that keeps SMs busy for long; otherwise such waits can run
+ *   out and the call reports NVFP4_MOE_ERR_TIMEOUT.
  *
  * Threading: a handle may be used from one host thread at a time. Two forward
  *   calls that run concurrently on the GPU must not share a workspace.
@@ -168,9 +178,9 @@ typedef struct {
 } nvfp4_moe_io;
 
 /* Validates dims and weight pointers (all checks before any allocation), then
- * allocates the handle and its 64-byte device status block on the current device.
- * On failure *out is set to NULL and nothing stays allocated. Requires an sm_100
- * device to be current. */
+ * allocates the handle, its device status block and decode state on the current
+ * device. On failure *out is set to NULL and nothing stays allocated. Requires
+ * an sm_100 device to be current. */
 NVFP4_MOE_API int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
                      const nvfp4_moe_weights *weights);
 
@@ -186,7 +196,8 @@ NVFP4_MOE_API int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void
                       size_t workspace_bytes, void *stream);
 
 /* Synchronises `stream`, returns the first device-side error latched since the
- * last call (0 if none) and clears it. */
+ * last call (0 if none) and clears it. After an error it also clears the decode
+ * state a launch that gave up may have left behind. */
 NVFP4_MOE_API int nvfp4_moe_get_status(nvfp4_moe_t *h, void *stream);
 
 /* Phase timing (optional): when n_events == NVFP4_MOE_PHASE_EVENTS and events
@@ -206,19 +217,20 @@ NVFP4_MOE_API int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events
  * for callers that cannot allocate device memory at all, and so cannot create a
  * handle -- nvfp4_moe_create allocates a status block -- or pass a workspace).
  * It runs the same decode path as nvfp4_moe_forward for 1 <= T <= 8 tokens, with
- * its scratch in a 1 MiB array compiled into the library (a file-scope
+ * its scratch in a 2 MiB array compiled into the library (a file-scope
  * __device__ array: every GPU that loads the library holds it until the process
  * exits). dims and weights are checked exactly as by nvfp4_moe_create; io and
  * stream are as for nvfp4_moe_forward. Calls no cudaMalloc/cudaFree.
  *   - T > 8 returns NVFP4_MOE_ERR_UNSUPPORTED_DIMS; a layer whose decode
- *     scratch for this T exceeds 1 MiB - 256 bytes returns
+ *     scratch and state for this T exceed 2 MiB - 256 bytes returns
  *     NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL (e.g. H = I = 8192 with K = 16). Both
  *     are checked before anything is enqueued. T = 0 is a no-op.
  *   - The first call on a device looks up the array's device address on that
  *     device (cudaGetSymbolAddress); make that first call before any stream
  *     capture on the device.
  *   - All calls on a device share the one array, which keeps the last call's
- *     contents; each call clears what must start at zero. Calls that overlap on
+ *     contents; each call clears what must start at zero (the status words and
+ *     the decode state, with one cudaMemsetAsync). Calls that overlap on
  *     the GPU (different streams, or other threads) race on it: serialise them.
  *   - Device-side routing problems (bad precomputed ids, non-finite logits) are
  *     contained exactly as in nvfp4_moe_forward but cannot be read back: there
@@ -227,7 +239,8 @@ NVFP4_MOE_API int nvfp4_moe_forward_decode_static(const nvfp4_moe_dims *dims,
                                                   const nvfp4_moe_weights *weights,
                                                   const nvfp4_moe_io *io, void *stream);
 
-/* Frees the handle and its status block. Never touches the borrowed weights. */
+/* Frees the handle, its status block and decode state. Never touches the
+ * borrowed weights. */
 NVFP4_MOE_API void nvfp4_moe_destroy(nvfp4_moe_t *h);
 
 /* Static string for a status code. */
