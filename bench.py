@@ -258,37 +258,72 @@ def run_ours(args, ws, rank, local):
                                                  torch.linalg.vector_norm(ob.double())), 5)
         del xf, ob, oi
 
-    # ---- end to end: host buffers, copies inside the timed region
+    # ---- end to end: host buffers, copies inside the timed region. Every step
+    # copies its inputs from pinned host memory and reads its output back; the
+    # copies of neighbouring steps overlap the layer (H2D, compute and D2H on
+    # three streams, two device input/output buffers, events guarding reuse),
+    # as a serving loop would run it.
     if not args.no_e2e:
         xh = x.cpu().pin_memory()
         lh = logits.cpu().pin_memory()
         xsh = xs.cpu().pin_memory() if xs is not None else None
-        oh = torch.empty(T, d.H, dtype=torch.float32).pin_memory()
-        xd, ld_ = torch.empty_like(x), torch.empty_like(logits)
-        xsd = torch.empty_like(xs) if xs is not None else None
+        ohs = [torch.empty(T, d.H, dtype=torch.float32).pin_memory() for _ in range(2)]
+        xds = [torch.empty_like(x) for _ in range(2)]
+        lds = [torch.empty_like(logits) for _ in range(2)]
+        xsds = [torch.empty_like(xs) if xs is not None else None for _ in range(2)]
+        outs = [out, torch.empty_like(out)]
+        m.set_phase_events(())      # no per-phase records in this loop
+        # one workspace: every forward runs on the compute stream, one at a time
+        s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()
+        in_ready = [ev(), ev()]     # inputs of buffer b copied
+        in_free = [ev(), ev()]      # compute done reading inputs of buffer b
+        out_ready = [ev(), ev()]    # output of buffer b computed
+        out_free = [ev(), ev()]     # output of buffer b copied back
+        for e_ in in_free + out_free:
+            e_.record(torch.cuda.current_stream())
 
-        def e2e_step():
-            xd.copy_(xh, non_blocking=True)
-            ld_.copy_(lh, non_blocking=True)
-            if xsd is not None:
-                xsd.copy_(xsh, non_blocking=True)
-            m.forward(xd, logits=ld_, x_scale=xsd, out=out, workspace=ws_buf)
-            oh.copy_(out, non_blocking=True)
+        def e2e_step(i):
+            bb = i & 1
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(in_free[bb])
+                xds[bb].copy_(xh, non_blocking=True)
+                lds[bb].copy_(lh, non_blocking=True)
+                if xsh is not None:
+                    xsds[bb].copy_(xsh, non_blocking=True)
+                in_ready[bb].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(in_ready[bb])
+                s_cmp.wait_event(out_free[bb])
+                m.forward(xds[bb], logits=lds[bb], x_scale=xsds[bb], out=outs[bb], workspace=ws_buf,
+                          stream=s_cmp)
+                in_free[bb].record(s_cmp)
+                out_ready[bb].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(out_ready[bb])
+                ohs[bb].copy_(outs[bb], non_blocking=True)
+                out_free[bb].record(s_out)
 
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
+        for i in range(max(1, args.warmup)):
+            e2e_step(i)
         torch.cuda.synchronize()
         barrier(ws)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(args.steps):
-            e2e_step()
-        b.record()
+        a.record(s_in)
+        for i in range(args.steps):
+            e2e_step(i)
+        s_in.wait_stream(s_out)
+        b.record(s_in)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(b), ws)
+        st = m.status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} after the end-to-end steps")
         h2d = xh.numel() * xh.element_size() + lh.numel() * 4 + (xsh.numel() * 4 if xsh is not None else 0)
         res["e2e"] = {"value": round(ws * T * args.steps / (e_ms / 1e3), 1), "unit": "tok/s",
-                      "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(oh.numel() * 4)}
+                      "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(ohs[0].numel() * 4),
+                      "ms_per_step": round(e_ms / args.steps, 4),
+                      "schedule": "H2D, layer and D2H on three streams, double-buffered across steps"}
         res["gpu_launches"] += 8 * args.steps
 
     # ---- decode expert GB/s (8 distinct layers so the L2 never holds the weights)
