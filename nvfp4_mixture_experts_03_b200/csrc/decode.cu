@@ -26,7 +26,8 @@
 //     h rows into shared memory, and adds its partial sums into out.
 // No grid-wide barrier: the only cross-CTA waits are the per-expert ready counts
 // and one count of CTAs that have read the activations (out may alias them),
-// all bounded. The last CTA to finish resets the counts for the next launch.
+// all bounded. The last CTA past its waits resets the counts, at its end, for
+// the next launch.
 // Arithmetic: each weight is decoded exactly to F16 (E2M1 -> F16 conversion
 // times its E4M3 group scale: at most 6 significant bits, exact in F16) and fed
 // to mma.sync m16n8k16 with the token slots as N, FP32 accumulation; the tensor
@@ -493,7 +494,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     int x1 = a1;
     const Chunk c1 = take_chunk(x1, b1, R1);
     PassBuf buf0, buf1;
-    issue_loads<0>(p, item_of<0>(p, R, c1), lane >> 2, lane & 3, c1.r0, c1.r1, buf0);
 
     // per-token amax -> power-of-two shift -> F16 activations in shared memory
     // (token slots past T are zeros)
@@ -560,6 +560,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
         atomicAdd(ds + kDsStaged, 1);
     }
 
+    // first weight loads after the staging: the fence above then has no weight
+    // loads of its own thread to wait for
+    issue_loads<0>(p, item_of<0>(p, R, c1), lane >> 2, lane & 3, c1.r0, c1.r1, buf0);
     run_range<0>(p, R, S, x1, b1, c1, buf0, buf1, 0);
 
     // phase 2: this CTA's share, split evenly over its warps
@@ -577,11 +580,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     const int pos_lo = u_hi >= u_lo ? R.uoff[u_lo] : 0;
     const int rows = u_hi >= u_lo ? R.uoff[u_hi + 1] - pos_lo : 0;
     __syncthreads();
-    if (threadIdx.x == 0 && u_hi >= u_lo) {
-        bool ok = wait_geq(ds + kDsStaged, gridDim.x, p.status, 101);
-        for (int u = u_lo; ok && u <= u_hi; u++) ok = wait_geq(ds + kDsReady + u, I / 8, p.status, 102);
-        if (rows > p.dec_hs_rows) latch_status(p.status, NVFP4_MOE_ERR_UNSUPPORTED_DIMS, 103);
-        __threadfence();
+    // This CTA's last use of the counts is the wait below; once every CTA has
+    // passed it, every count is final (each used expert has down items, so its
+    // gate/up items are all finished), and the last CTA to arrive resets them.
+    // The arrival is issued right after the wait and its result is consumed at
+    // the end, so its round trip hides behind the down work.
+    int exit_prev = 0;
+    if (threadIdx.x == 0) {
+        if (u_hi >= u_lo) {
+            bool ok = wait_geq(ds + kDsStaged, gridDim.x, p.status, 101);
+            for (int u = u_lo; ok && u <= u_hi; u++) ok = wait_geq(ds + kDsReady + u, I / 8, p.status, 102);
+            if (rows > p.dec_hs_rows) latch_status(p.status, NVFP4_MOE_ERR_UNSUPPORTED_DIMS, 103);
+            __threadfence();
+        }
+        exit_prev = atomicAdd(ds + kDsExit, 1);
     }
     __syncthreads();
     {
@@ -595,17 +607,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     __syncthreads();
     if (rows <= p.dec_hs_rows) run_range<1>(p, R, S, x2, b2, c2, buf0, buf1, pos_lo);
 
-    // The next layer's grid may launch once every CTA is here; the last CTA to
-    // finish resets the counts for the next launch.
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        if (atomicAdd(ds + kDsExit, 1) == (int)gridDim.x - 1) {
-            for (int u = 0; u < U; u++) ds[kDsReady + u] = 0;
-            ds[kDsStaged] = 0;
-            __threadfence();
-            ds[kDsExit] = 0;
-        }
+    // The next layer's grid may launch once every CTA is here.
+    if (threadIdx.x == 0 && exit_prev == (int)gridDim.x - 1) {
+        for (int u = 0; u < U; u++) ds[kDsReady + u] = 0;
+        ds[kDsStaged] = 0;
+        ds[kDsExit] = 0;
     }
     asm volatile("griddepcontrol.launch_dependents;" :::);
 }
