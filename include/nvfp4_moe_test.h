@@ -1,0 +1,39 @@
+/*
+ * Test hooks of the NVFP4 MoE layer library (libnvfp4_moe.so).
+ *
+ * The pages have no counterpart: these exist only so that the library's own
+ * fault tests can drive its error paths without faulting, trapping or hanging
+ * a GPU. Production code never calls them; with the hooks off (the default)
+ * the library behaves exactly as nvfp4_moe.h describes.
+ */
+#ifndef NVFP4_MOE_TEST_H
+#define NVFP4_MOE_TEST_H
+
+#include "nvfp4_moe.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Decode (T <= 8): CTA 0 never reports that it has read the activations, so
+ * every CTA's bounded wait before the down phase runs out (after about 200 ms),
+ * the call latches NVFP4_MOE_ERR_TIMEOUT, and the layer's output is not valid.
+ * nvfp4_moe_get_status then returns TIMEOUT and clears the decode state, after
+ * which calls with the flag off are correct again. */
+#define NVFP4_MOE_TEST_DECODE_STALL 1
+
+/* Sets the test flags of a handle (0 = none). Returns NVFP4_MOE_OK, or
+ * NVFP4_MOE_ERR_INVALID_ARG for a NULL handle or an unknown flag. */
+NVFP4_MOE_API int nvfp4_moe_test_set_flags(nvfp4_moe_t *h, int32_t flags);
+
+/* Makes the n-th device allocation (counting from 1) made by later
+ * nvfp4_moe_create calls fail as if the device were out of memory; the hook
+ * then disarms itself. n <= 0 disarms it. create must then return
+ * NVFP4_MOE_ERR_CUDA with nothing left allocated. Process-wide; not
+ * thread-safe. */
+NVFP4_MOE_API void nvfp4_moe_test_fail_alloc(int32_t n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -27,11 +27,13 @@ OUT_F32, OUT_F32_ADD = 0, 1
 DECODE_MAX_T = 8
 MAX_TOPK = 16
 
-# Every function the header declares (checked against include/nvfp4_moe.h by the tests).
+# Every function the headers declare (checked against include/*.h by the tests).
 EXPORTS = ("nvfp4_moe_create", "nvfp4_moe_workspace_bytes", "nvfp4_moe_forward",
            "nvfp4_moe_get_status", "nvfp4_moe_destroy", "nvfp4_moe_strerror",
            "nvfp4_moe_abi_version", "nvfp4_moe_set_phase_events",
-           "nvfp4_moe_forward_decode_static")
+           "nvfp4_moe_forward_decode_static",
+           "nvfp4_moe_test_set_flags", "nvfp4_moe_test_fail_alloc")
+TEST_DECODE_STALL = 1   # include/nvfp4_moe_test.h
 PHASE_EVENTS = 5
 
 
@@ -137,6 +139,17 @@ def nvfp4_moe_set_phase_events(handle: int, events) -> int:
     """events: sequence of PHASE_EVENTS cudaEvent_t handles (ints), or () to turn off."""
     arr = (C.c_void_p * max(1, len(events)))(*[C.c_void_p(int(e)) for e in events])
     return lib().nvfp4_moe_set_phase_events(C.c_void_p(handle), arr, len(events))
+
+
+def nvfp4_moe_test_set_flags(handle: int, flags: int) -> int:
+    """Test hook (include/nvfp4_moe_test.h): TEST_DECODE_STALL makes decode's bounded
+    waits run out, so the call latches TIMEOUT."""
+    return lib().nvfp4_moe_test_set_flags(C.c_void_p(handle), C.c_int32(flags))
+
+
+def nvfp4_moe_test_fail_alloc(n: int) -> None:
+    """Test hook: the n-th device allocation of later creates fails (then disarms)."""
+    lib().nvfp4_moe_test_fail_alloc(C.c_int32(n))
 
 
 def nvfp4_moe_forward_decode_static(dims: Dims, weights: Weights, io: IO, stream: int) -> int:

@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include "nvfp4_moe.h"
+#include "nvfp4_moe_test.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "this library targets sm_100a only"
@@ -90,6 +91,7 @@ struct Params {
     int32_t *dstate;           // decode: counters (kDs*), zero between launches
     float *dgu;                // decode: [pairs][2][I] FP32 partial sums, zero between launches
     int32_t dec_hs_rows;       // decode: h rows one CTA stages for its down range
+    int32_t test_flags;        // NVFP4_MOE_TEST_* (test hooks; 0 in production)
 };
 
 constexpr int kActF32 = 2;     // internal: act is FP32, rounded to BF16 first

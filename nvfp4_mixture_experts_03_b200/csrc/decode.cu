@@ -555,7 +555,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     __syncthreads();
     // the activations are read and this stripe of out is cleared: phase-2 adds
     // anywhere into out wait for every CTA to get here (out may alias act)
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && !((p.test_flags & NVFP4_MOE_TEST_DECODE_STALL) && blockIdx.x == 0)) {
         __threadfence();
         atomicAdd(ds + kDsStaged, 1);
     }

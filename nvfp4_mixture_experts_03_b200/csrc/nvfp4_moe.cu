@@ -29,6 +29,7 @@ struct nvfp4_moe {
     uint8_t *dstate;  // decode state (zero between launches), for dec_pairs pairs
     size_t dstate_bytes;
     int dec_pairs;
+    int32_t test_flags;  // NVFP4_MOE_TEST_* (test hooks)
     cudaEvent_t phase[NVFP4_MOE_PHASE_EVENTS];
     bool phase_on;
 };
@@ -84,6 +85,16 @@ bool make_map_codes(CUtensorMap *m, const void *base, int64_t rows, int64_t cols
 }
 
 inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Test hook: the n-th device allocation of later creates fails (then disarms).
+int g_fail_alloc = 0;
+cudaError_t dev_alloc(void **p, size_t bytes) {
+    if (g_fail_alloc > 0 && --g_fail_alloc == 0) {
+        *p = nullptr;
+        return cudaErrorMemoryAllocation;
+    }
+    return cudaMalloc(p, bytes);
+}
 inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 inline bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
 
@@ -202,13 +213,14 @@ int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
     h->status = nullptr;
     h->dstate = nullptr;
     h->phase_on = false;
+    h->test_flags = 0;
     const int dec_t = d.max_tokens < NVFP4_MOE_DECODE_MAX_T ? d.max_tokens : NVFP4_MOE_DECODE_MAX_T;
     h->dec_pairs = dec_t * d.top_k;
     h->dstate_bytes = h->dec_pairs > 0 ? decode_state_bytes(h->dec_pairs, d.inter) : 0;
-    if (cudaMalloc(&h->status, kStatusWords * sizeof(int32_t)) != cudaSuccess ||
+    if (dev_alloc(reinterpret_cast<void **>(&h->status), kStatusWords * sizeof(int32_t)) != cudaSuccess ||
         cudaMemset(h->status, 0, kStatusWords * sizeof(int32_t)) != cudaSuccess ||
         (h->dstate_bytes &&
-         (cudaMalloc(&h->dstate, h->dstate_bytes) != cudaSuccess ||
+         (dev_alloc(reinterpret_cast<void **>(&h->dstate), h->dstate_bytes) != cudaSuccess ||
           cudaMemset(h->dstate, 0, h->dstate_bytes) != cudaSuccess))) {
         if (h->status) cudaFree(h->status);
         if (h->dstate) cudaFree(h->dstate);
@@ -300,6 +312,7 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     p.nch = L.nch;
     p.max_tiles_gu = L.max_gu;
     p.max_tiles_dn = L.max_dn;
+    p.test_flags = h->test_flags;
     if (T <= NVFP4_MOE_DECODE_MAX_T) {
         if (T * d.top_k > h->dec_pairs || !h->dstate) return NVFP4_MOE_ERR_INVALID_ARG;
         p.dstate = reinterpret_cast<int32_t *>(h->dstate);
@@ -377,6 +390,14 @@ int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events, int32_t n_ev
     h->phase_on = true;
     return NVFP4_MOE_OK;
 }
+
+int nvfp4_moe_test_set_flags(nvfp4_moe_t *h, int32_t flags) {
+    if (!h || (flags & ~NVFP4_MOE_TEST_DECODE_STALL)) return NVFP4_MOE_ERR_INVALID_ARG;
+    h->test_flags = flags;
+    return NVFP4_MOE_OK;
+}
+
+void nvfp4_moe_test_fail_alloc(int32_t n) { g_fail_alloc = n > 0 ? n : 0; }
 
 void nvfp4_moe_destroy(nvfp4_moe_t *h) {
     if (!h) return;
@@ -479,6 +500,7 @@ int nvfp4_moe_forward_decode_static(const nvfp4_moe_dims *dims, const nvfp4_moe_
     h.device = dev;
     h.num_sms = sms;
     h.pf_clusters = 0;   // T <= 8 never reaches the prefill GEMMs
+    h.test_flags = 0;
     h.status = reinterpret_cast<int32_t *>(scratch);
     h.dstate = scratch + kStaticStatusBytes;
     h.dstate_bytes = state;

@@ -10,13 +10,16 @@ import pytest
 import nvfp4_mixture_experts_03_b200 as nv
 from conftest import ROOT
 
-HEADER = os.path.join(ROOT, "include", "nvfp4_moe.h")
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
 
 
 def declared_functions():
-    src = open(HEADER).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(nvfp4_moe_\w+)\s*\(", src)))
+    names = set()
+    for h in HEADERS:
+        src = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(nvfp4_moe_\w+)\s*\(", src))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")
