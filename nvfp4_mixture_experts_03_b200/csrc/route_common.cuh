@@ -16,6 +16,12 @@ __device__ inline uint32_t sel_key(float v) {
     return k < 2u ? 2u : k;  // -inf maps to 0x007FFFFF, so this never changes a number's order
 }
 
+// The logit a key came from (exact for every non-NaN key; +0 for the merged
+// zeros; a NaN for the NaN key).
+__device__ inline float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // One warp selects the top-K of one token's logits (E <= 32*NPER): K rounds of
 // (per-lane argmax over its NPER keys, warp max of the key, warp min of the
 // expert id among lanes holding it), so equal logits go to the lower id. Lane
@@ -24,12 +30,11 @@ template <int NPER>
 __device__ inline void warp_topk(const float *__restrict__ row, int E, int K, int lane,
                                  int &my_id, float &my_w, bool &finite) {
     uint32_t key[NPER];
-    float val[NPER];
     // all loads first (clamped in-bounds addresses), so they are in flight together
 #pragma unroll
-    for (int i = 0; i < NPER; i++) val[i] = __ldg(row + min(lane + 32 * i, E - 1));
+    for (int i = 0; i < NPER; i++) key[i] = __float_as_uint(__ldg(row + min(lane + 32 * i, E - 1)));
 #pragma unroll
-    for (int i = 0; i < NPER; i++) key[i] = (lane + 32 * i < E) ? sel_key(val[i]) : 0u;
+    for (int i = 0; i < NPER; i++) key[i] = (lane + 32 * i < E) ? sel_key(__uint_as_float(key[i])) : 0u;
     my_id = 0;
     float my_v = 0.0f;
     for (int j = 0; j < K; j++) {
@@ -42,13 +47,9 @@ __device__ inline void warp_topk(const float *__restrict__ row, int E, int K, in
         const uint32_t cand = (best == gmax) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
         const int e = (int)__reduce_min_sync(0xffffffffu, cand);
         const int hit = ((e & 31) == lane) ? (e >> 5) : -1;
-        float v = 0.0f;
 #pragma unroll
-        for (int i = 0; i < NPER; i++) {
-            v = (i == hit) ? val[i] : v;
-            key[i] = (i == hit) ? 0u : key[i];
-        }
-        v = __shfl_sync(0xffffffffu, v, e & 31);
+        for (int i = 0; i < NPER; i++) key[i] = (i == hit) ? 0u : key[i];
+        const float v = key_value(gmax);   // the selected logit, known to every lane
         if (lane == j) {
             my_id = e;
             my_v = v;
