@@ -246,17 +246,6 @@ __device__ inline void tma_prefetch_desc(const CUtensorMap *map) {
 }
 
 // ----------------------------------------------------------------- tcgen05
-__device__ inline void tmem_alloc(uint32_t *slot_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(slot_smem)),
-                 "r"(ncols));
-}
-__device__ inline void tmem_relinquish() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-}
-__device__ inline void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
-}
 // Pair forms (cta_group::2): one warp with the same warp index in each CTA of the
 // pair issues alloc / relinquish / dealloc; the same columns are taken in both.
 __device__ inline void tmem_alloc_pair(uint32_t *slot_smem, uint32_t ncols) {
@@ -275,14 +264,6 @@ __device__ inline void tc_fence_before() {
 }
 __device__ inline void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-// D[tmem] (+)= A[smem desc] x B[smem desc]^T, kind::f16 (both operands F16), one CTA.
-__device__ inline void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                  uint32_t accumulate) {
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 // Pair MMA (issued by the leader CTA only): M = 256 rows, the first 128 from the
 // leader's A tile and TMEM, the next 128 from the peer's; B's first N/2 rows from
@@ -306,13 +287,6 @@ __device__ inline void tc_commit_pair_mc(uint64_t *bar, uint16_t cta_mask) {
 __device__ inline void tc_commit_pair(uint64_t *bar) {
     asm volatile(
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-// Arrives on `bar` once every tcgen05.mma issued so far by this thread has completed.
-__device__ inline void tc_commit(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             smem_u32(bar))
         : "memory");
 }

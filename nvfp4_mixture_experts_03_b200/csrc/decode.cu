@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     int32_t *ds = p.dstate;
 
     // Everything this layer reads may come from the previous kernel in the stream.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    grid_dep_wait();
 
     // the activations first: their loads are then not queued behind the weights'
     const int raw_bytes = T * raw_act_bytes(p.act_type, H);
@@ -613,7 +613,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
         ds[kDsStaged] = 0;
         ds[kDsExit] = 0;
     }
-    asm volatile("griddepcontrol.launch_dependents;" :::);
+    grid_dep_launch();
 }
 
 static int sm_count() {
