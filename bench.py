@@ -143,6 +143,11 @@ def cpu_oracle_rate(layer_cpu, x, logits, K, n_tokens, x_scale=None):
     return n_tokens / dt, dt
 
 
+def oracle_threads(n_tokens):
+    """Worker threads the C oracle starts for n sampled tokens: one per online CPU, at most one per token."""
+    return max(1, min(n_tokens, os.cpu_count() or 1))
+
+
 # ------------------------------------------------------------------- workloads
 
 def make_prefill(wl_name, dev):
@@ -338,7 +343,7 @@ def run_ours(args, ws, rank, local):
         rate, dt = cpu_oracle_rate(layer_cpu, xc, lc, d.K, 8, xsc)       # calibrate
         n = int(min(T, max(8, rate * args.cpu_seconds)))
         rate, dt = cpu_oracle_rate(layer_cpu, xc, lc, d.K, n, xsc)
-        res["cpu_baseline"] = {"value": round(rate, 3), "unit": "tok/s", "cores": os.cpu_count(),
+        res["cpu_baseline"] = {"value": round(rate, 3), "unit": "tok/s", "cores": oracle_threads(n),
                                "kind": "oracle",
                                "sample": f"first {n} of the {T} tokens of the same chunk, FP64, "
                                          f"{dt:.1f} s wall"}
@@ -565,7 +570,7 @@ def run_reference(args, ws, rank):
             "ms_per_step": round(dt * 1e3 / args.steps, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{wl.name}: {wl.note}", "tokens_per_step": n},
-            "cpu_baseline": {"value": round(v, 3), "unit": "tok/s", "cores": os.cpu_count(),
+            "cpu_baseline": {"value": round(v, 3), "unit": "tok/s", "cores": oracle_threads(n),
                              "kind": "oracle",
                              "sample": f"first {n} tokens of the {T}-token chunk per step"
                                        + (", one layer; rate divided by 48 layers" if per_layers > 1 else "")},
