@@ -165,6 +165,28 @@ __device__ inline bool epi_all(bool v) {
     return r != 0;
 }
 
+// Copies a staged chunk (ncol columns of kRowsB F16 values, each column contiguous
+// in shared memory) to `ncol` rows of `dst` (row stride `ld` elements), by the 128
+// epilogue threads with 16-byte accesses. Every shared load is issued before the
+// first global store: the compiler cannot tell the two apart and would otherwise
+// wait for each store before the next load.
+template <int kRowsB>
+__device__ inline void store_chunk(const __half *stage, __half *dst, size_t ld, int ncol) {
+    constexpr int kParts = kRowsB / 8, kPer = 32 * kParts / 128;
+    const int nq = ncol * kParts;
+    uint4 val[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; k++) {
+        const int q = threadIdx.x + 128 * k;
+        if (q < nq) val[k] = reinterpret_cast<const uint4 *>(stage)[q];
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; k++) {
+        const int q = threadIdx.x + 128 * k;
+        if (q < nq) reinterpret_cast<uint4 *>(dst + (size_t)(q / kParts) * ld)[q % kParts] = val[k];
+    }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const Params p, const __grid_constant__ CUtensorMap map_b,
@@ -451,6 +473,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < kChunks; c++) {
                     if (32 * c >= t.ntok) break;
                     __half *hs = reinterpret_cast<__half *>(epi_stage) + (c & 1) * (32 * kGuCta);
+                    // This lane's 16 column factors, in registers before the first
+                    // staging store (shared loads after it would wait for it).
+                    const int cj0 = is_gate ? 0 : 16;
+                    float xs[16];
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        const float4 f = reinterpret_cast<const float4 *>(colf_s + 32 * c + cj0)[k];
+                        xs[4 * k] = f.x; xs[4 * k + 1] = f.y; xs[4 * k + 2] = f.z; xs[4 * k + 3] = f.w;
+                    }
                     uint32_t v[32];
                     tmem_ld32(tbase + 32 * c, v);
                     tmem_ld_wait();
@@ -462,18 +493,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
                         const float gacc = is_gate ? mine_lo : recv;
                         const float uacc = is_gate ? recv : mine_hi;
-                        const int cj = j + (is_gate ? 0 : 16);
-                        const float xs = colf_s[32 * c + cj];
-                        const float gv = gacc * sg * xs, uv = uacc * su * xs;
-                        hs[cj * kGuCta + il] = __float2half_rn(silu(gv) * uv);
+                        const float gv = gacc * sg * xs[j], uv = uacc * su * xs[j];
+                        hs[(cj0 + j) * kGuCta + il] = __float2half_rn(silu(gv) * uv);
                     }
                     epi_sync();
-                    const int ncol = min(32, t.ntok - 32 * c);
-                    for (int q = threadIdx.x; q < ncol * (kGuCta / 8); q += 128) {
-                        const int col = q / (kGuCta / 8), part = q % (kGuCta / 8);
-                        const uint4 val = reinterpret_cast<const uint4 *>(hs + col * kGuCta)[part];
-                        reinterpret_cast<uint4 *>(p.h + (size_t)(t.pos0 + 32 * c + col) * p.I + i0)[part] = val;
-                    }
+                    store_chunk<kGuCta>(hs, p.h + (size_t)(t.pos0 + 32 * c) * p.I + i0, p.I,
+                                        min(32, t.ntok - 32 * c));
                 }
             } else {
                 // y * s_d * w staged as [32 columns][128 hidden rows] F16, written into
@@ -486,19 +511,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < kChunks; c++) {
                         if (32 * c >= t.ntok) break;
                         __half *ys = reinterpret_cast<__half *>(epi_stage) + (c & 1) * (32 * kBM);
+                        // The chunk's 32 column factors in registers before the first
+                        // staging store.
+                        float cf[32];
+#pragma unroll
+                        for (int k = 0; k < 8; k++) {
+                            const float4 f = reinterpret_cast<const float4 *>(colf_s + 32 * c)[k];
+                            cf[4 * k] = f.x; cf[4 * k + 1] = f.y; cf[4 * k + 2] = f.z; cf[4 * k + 3] = f.w;
+                        }
                         uint32_t v[32];
                         tmem_ld32(tbase + 32 * c, v);
                         tmem_ld_wait();
 #pragma unroll
                         for (int j = 0; j < 32; j++)
-                            ys[j * kBM + r] = __float2half_rn(__uint_as_float(v[j]) * colf_s[32 * c + j]);
+                            ys[j * kBM + r] = __float2half_rn(__uint_as_float(v[j]) * cf[j]);
                         epi_sync();
-                        const int ncol = min(32, t.ntok - 32 * c);
-                        for (int q = threadIdx.x; q < ncol * (kBM / 8); q += 128) {
-                            const int col = q / (kBM / 8), part = q % (kBM / 8);
-                            const uint4 val = reinterpret_cast<const uint4 *>(ys + col * kBM)[part];
-                            reinterpret_cast<uint4 *>(p.xh + (size_t)(t.pos0 + 32 * c + col) * p.H + m)[part] = val;
-                        }
+                        store_chunk<kBM>(ys, p.xh + (size_t)(t.pos0 + 32 * c) * p.H + m, p.H,
+                                         min(32, t.ntok - 32 * c));
                     }
                 }
             }
