@@ -616,7 +616,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     grid_dep_launch();
 }
 
-static int sm_count() {
+int sm_count() {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -221,13 +221,15 @@ __global__ void __launch_bounds__(256) prep_prefill_kernel(Params p) {
 
 // out_t (+)= sum_j yp[pos(t, j)] over the token's K pairs, in the fixed order
 // j = 0..K-1 with FP32 accumulation (yp holds w * s_d * y per pair, F16, in the
-// buffer that held the pair-ordered activations). One CTA per token; each thread
-// issues all K loads of its 8 columns before adding them up.
+// buffer that held the pair-ordered activations). Resident CTAs stride over the
+// tokens (one launch wave, no per-token CTA start-up); each thread issues all K
+// loads of its 8 columns before adding them up.
 __global__ void __launch_bounds__(256) combine_kernel(Params p) {
-    const int t = blockIdx.x;
-    __shared__ int spos[NVFP4_MOE_MAX_TOPK];
-    if (threadIdx.x < p.K) spos[threadIdx.x] = p.inv[(size_t)t * p.K + threadIdx.x];
-    __syncthreads();
+  for (int t = blockIdx.x; t < p.T; t += gridDim.x) {
+    int spos[NVFP4_MOE_MAX_TOPK];
+#pragma unroll
+    for (int j = 0; j < NVFP4_MOE_MAX_TOPK; j++)
+        if (j < p.K) spos[j] = __ldg(p.inv + (size_t)t * p.K + j);
     for (int k8 = threadIdx.x; k8 < p.H / 8; k8 += blockDim.x) {
         uint4 y[NVFP4_MOE_MAX_TOPK];
 #pragma unroll
@@ -261,6 +263,7 @@ __global__ void __launch_bounds__(256) combine_kernel(Params p) {
         o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
         o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
+  }
 }
 
 // ------------------------------------------------------------------ launch
@@ -289,8 +292,12 @@ void launch_prep_prefill(const Params &p, cudaStream_t s) {
     prep_prefill_kernel<<<p.T, 256, 0, s>>>(p);
 }
 
+int sm_count();   // SMs of the current device (decode.cu)
+
 void launch_combine(const Params &p, cudaStream_t s) {
-    combine_kernel<<<p.T, 256, 0, s>>>(p);
+    // eight 256-thread CTAs per SM (the SM's 2048 threads), fewer for short batches
+    const int resident = 8 * sm_count();
+    combine_kernel<<<p.T < resident ? p.T : resident, 256, 0, s>>>(p);
 }
 
 
