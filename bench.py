@@ -143,6 +143,19 @@ def cpu_oracle_rate(layer_cpu, x, logits, K, n_tokens, x_scale=None):
     return n_tokens / dt, dt
 
 
+def cpu_model():
+    """The host CPU's model name, as the kernel reports it."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def oracle_threads(n_tokens):
     """Worker threads the C oracle starts for n sampled tokens: one per online CPU, at most one per token."""
     return max(1, min(n_tokens, os.cpu_count() or 1))
@@ -350,7 +363,7 @@ def run_ours(args, ws, rank, local):
         n = int(min(T, max(8, rate * args.cpu_seconds)))
         rate, dt = cpu_oracle_rate(layer_cpu, xc, lc, d.K, n, xsc)
         res["cpu_baseline"] = {"value": round(rate, 3), "unit": "tok/s", "cores": oracle_threads(n),
-                               "kind": "oracle",
+                               "cpu_model": cpu_model(), "kind": "oracle",
                                "sample": f"first {n} of the {T} tokens of the same chunk, FP64, "
                                          f"{dt:.1f} s wall"}
     m.close()
@@ -582,7 +595,7 @@ def run_reference(args, ws, rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{wl.name}: {wl.note}", "tokens_per_step": n},
             "cpu_baseline": {"value": round(v, 3), "unit": "tok/s", "cores": oracle_threads(n),
-                             "kind": "oracle",
+                             "cpu_model": cpu_model(), "kind": "oracle",
                              "sample": f"first {n} tokens of the {T}-token chunk per step"
                                        + (", one layer; rate divided by 48 layers" if per_layers > 1 else "")},
             "e2e": {"value": round(v, 3), "unit": "tok/s", "h2d_bytes_per_step": 0,
