@@ -143,6 +143,21 @@ def cpu_oracle_rate(layer_cpu, x, logits, K, n_tokens, x_scale=None):
     return n_tokens / dt, dt
 
 
+def oracle_baseline(layer_cpu, x, logits, K, T, seconds, x_scale=None, layers=1):
+    """The bench line's `cpu_baseline`: the oracle on the first n tokens of the
+    chunk, n sized from an 8-token calibration to about `seconds` of CPU work.
+    `layers` > 1: one layer is timed and the rate divided by the layer count (the
+    stack's layers have one shape, so the oracle's cost per layer is the same)."""
+    rate, _ = cpu_oracle_rate(layer_cpu, x, logits, K, 8, x_scale)       # calibrate
+    n = int(min(T, max(8, rate * seconds)))
+    rate, dt = cpu_oracle_rate(layer_cpu, x, logits, K, n, x_scale)
+    sample = f"first {n} of the {T} tokens of the same chunk, FP64, {dt:.1f} s wall"
+    if layers > 1:
+        sample += f"; one layer timed, rate divided by {layers} layers (linear extrapolation)"
+    return {"value": round(rate / layers, 3), "unit": "tok/s", "cores": oracle_threads(n),
+            "cpu_model": cpu_model(), "kind": "oracle", "sample": sample}
+
+
 def cpu_model():
     """The host CPU's model name, as the kernel reports it."""
     try:
@@ -356,16 +371,9 @@ def run_ours(args, ws, rank, local):
 
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        layer_cpu = layer.to("cpu")
-        xc, lc = x.cpu(), logits.cpu()
-        xsc = xs.cpu() if xs is not None else None
-        rate, dt = cpu_oracle_rate(layer_cpu, xc, lc, d.K, 8, xsc)       # calibrate
-        n = int(min(T, max(8, rate * args.cpu_seconds)))
-        rate, dt = cpu_oracle_rate(layer_cpu, xc, lc, d.K, n, xsc)
-        res["cpu_baseline"] = {"value": round(rate, 3), "unit": "tok/s", "cores": oracle_threads(n),
-                               "cpu_model": cpu_model(), "kind": "oracle",
-                               "sample": f"first {n} of the {T} tokens of the same chunk, FP64, "
-                                         f"{dt:.1f} s wall"}
+        res["cpu_baseline"] = oracle_baseline(layer.to("cpu"), x.cpu(), logits.cpu(), d.K, T,
+                                              args.cpu_seconds,
+                                              xs.cpu() if xs is not None else None)
     m.close()
     return res
 
@@ -553,6 +561,11 @@ def run_stack(args, ws, rank, local):
         del g
     dec["peak"] = {"hbm_gbs": pk["hbm_gbs"], "source": pk_src}
     res["decode_stack"] = dec
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        # layer 0 on its own input bf16(x0), the stack's first step
+        res["cpu_baseline"] = oracle_baseline(layers[0].to("cpu"), x0.to(torch.bfloat16).cpu(),
+                                              lgp[0].cpu(), d.K, Tp, args.cpu_seconds,
+                                              layers=wl.layers)
     n_dec = sum(v["timed_launches"] for k, v in dec.items() if k.startswith("T"))
     res["gpu_launches"] += n_dec
     res["gpu_launches_by_region"]["decode_timed"] = n_dec

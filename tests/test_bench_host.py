@@ -50,3 +50,19 @@ def test_traffic_figure_only_while_sources_unchanged(tmp_path, monkeypatch):
     assert bench.profile_traffic("other", "w") is None
     (tmp_path / "k.cu").write_bytes(src + b"// changed\n")
     assert bench.profile_traffic("kern", "w") is None
+
+
+def test_oracle_baseline_sample_and_stack_label():
+    import synth
+    wl = synth.CONFIGS["tiny"]
+    seed = synth.workload_seed(wl)
+    layer = synth.make_layer(wl.dims, seed)
+    T = wl.tokens[0]
+    x = synth.make_x_bf16(T, wl.dims.H, seed)
+    logits = synth.make_logits(T, wl.dims.E, seed)
+    one = bench.oracle_baseline(layer, x, logits, wl.dims.K, T, 0.0)
+    assert one["kind"] == "oracle" and one["unit"] == "tok/s" and one["value"] > 0
+    assert one["sample"].startswith(f"first 8 of the {T} tokens") and one["cores"] == min(8, os.cpu_count())
+    many = bench.oracle_baseline(layer, x, logits, wl.dims.K, T, 0.0, layers=48)
+    assert "divided by 48 layers" in many["sample"]
+    assert 0 < many["value"] < one["value"]
