@@ -52,10 +52,21 @@
  * Errors: every call returns 0 (NVFP4_MOE_OK) or a negative nvfp4_moe_status.
  *   Host-side checks run before anything is enqueued; a call that fails them
  *   enqueues nothing. Conditions found on the device (routing id out of range
- *   or duplicated, a non-finite routing logit, a wait that gave up) are latched
- *   in the status block and returned by nvfp4_moe_get_status. forward never
- *   synchronises. Every device-side wait is bounded: a kernel whose wait runs
- *   out latches NVFP4_MOE_ERR_TIMEOUT and returns instead of hanging.
+ *   or duplicated, a non-finite routing logit, a non-finite computed value, a
+ *   wait that gave up) are latched in the status block and returned by
+ *   nvfp4_moe_get_status. forward never synchronises. Every device-side wait is
+ *   bounded: a kernel whose wait runs out latches NVFP4_MOE_ERR_TIMEOUT and
+ *   returns instead of hanging.
+ *
+ * Range: h = SiLU(g) * u is stored in F16 between the two projections, and the
+ *   grouped-GEMM path (T > 8) stores each pair's w * s_d * y row in F16 before the
+ *   FP32 combine. A value whose magnitude reaches 65520 there becomes inf; the
+ *   layer then latches NVFP4_MOE_ERR_NONFINITE (detail: stage and expert) rather
+ *   than return a silent inf. The tensor scales are applied in FP32 before these
+ *   roundings, never folded into F16 operands, so ordinary scales stay well
+ *   inside F16's normal range ("Strata NVFP4" README, "How it differs from
+ *   upstream Strata": folding a tiny scale into FP16 activations pushed them
+ *   into FP16 subnormals).
  *
  * Co-residency: the decode kernel (T <= 8) runs one CTA per SM and its CTAs wait
  *   on one another through counters (bounded). It assumes the GPU is not shared
@@ -98,7 +109,9 @@ typedef enum {
     NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL = -4,
     NVFP4_MOE_ERR_CUDA = -5,               /* a CUDA runtime/driver call failed           */
     NVFP4_MOE_ERR_BAD_ROUTING = -6,        /* device: precomputed id out of [0,E) or repeated */
-    NVFP4_MOE_ERR_NONFINITE = -7,          /* device: a selected routing logit is NaN/inf */
+    NVFP4_MOE_ERR_NONFINITE = -7,          /* device: a selected routing logit is NaN/inf, or a
+                                              computed h, per-pair down row or output value is
+                                              not finite (F16 intermediates overflowed)       */
     NVFP4_MOE_ERR_TIMEOUT = -8,            /* device: a bounded wait gave up              */
     NVFP4_MOE_ERR_NO_DEVICE = -9           /* no sm_100 device current                    */
 } nvfp4_moe_status;
@@ -180,12 +193,22 @@ typedef struct {
 /* Validates dims and weight pointers (all checks before any allocation), then
  * allocates the handle, its device status block and decode state on the current
  * device. On failure *out is set to NULL and nothing stays allocated. Requires
- * an sm_100 device to be current. */
+ * an sm_100 device to be current.
+ * Source: the pages' tensor readers validate the whole source before they
+ * allocate, refuse incomplete or ambiguous scale data and free what they
+ * allocated when an allocation fails ("TensorFold PR #906", first post); the
+ * handle borrows the caller's planes instead of copying them ("#1858 ...
+ * strata-safetensors", "Proposed contribution": bounded reads into buffers the
+ * caller owns). */
 NVFP4_MOE_API int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
                      const nvfp4_moe_weights *weights);
 
 /* Bytes of workspace a forward call with T tokens needs (256-byte aligned start
- * required). Returns 0 for a NULL handle or T outside [0, max_tokens]. */
+ * required). Returns 0 for a NULL handle or T outside [0, max_tokens].
+ * Source: every buffer of a forward call is the caller's, sized up front ("#1858
+ * ... strata-safetensors", "Proposed contribution": caller-owned bounded
+ * buffers); the workspace holds the routing arrays, the per-pair activation and
+ * h rows and the tile lists of the grouped GEMMs. */
 NVFP4_MOE_API size_t nvfp4_moe_workspace_bytes(const nvfp4_moe_t *h, int32_t T);
 
 /* Enqueues the whole layer on `stream` (a cudaStream_t; NULL = legacy default
@@ -197,7 +220,13 @@ NVFP4_MOE_API int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void
 
 /* Synchronises `stream`, returns the first device-side error latched since the
  * last call (0 if none) and clears it. After an error it also clears the decode
- * state a launch that gave up may have left behind. */
+ * state a launch that gave up may have left behind.
+ * Source: forward never waits on the host; the layer gathers each expert group
+ * into one launch after one wait ("Strata NVFP4" README, "How it differs from
+ * upstream Strata", the prompt-reading bullet), so device-side findings are
+ * read once, here, instead of after every launch; what is refused (bad routing,
+ * non-finite values) follows the readers' rule of refusing ambiguous or
+ * incomplete data rather than guessing ("TensorFold PR #906", first post). */
 NVFP4_MOE_API int nvfp4_moe_get_status(nvfp4_moe_t *h, void *stream);
 
 /* Phase timing (optional): when n_events == NVFP4_MOE_PHASE_EVENTS and events
@@ -225,9 +254,10 @@ NVFP4_MOE_API int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events
  *     scratch and state for this T exceed 2 MiB - 256 bytes returns
  *     NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL (e.g. H = I = 8192 with K = 16). Both
  *     are checked before anything is enqueued. T = 0 is a no-op.
- *   - The first call on a device looks up the array's device address on that
- *     device (cudaGetSymbolAddress); make that first call before any stream
- *     capture on the device.
+ *   - The first call on a device does a one-time set-up there: it looks up the
+ *     array's device address (cudaGetSymbolAddress) and opts the decode kernels
+ *     into the shared memory they need (cudaFuncSetAttribute). Make that first
+ *     call before any stream capture on the device.
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents; each call clears what must start at zero (the status words and
  *     the decode state, with one cudaMemsetAsync). Calls that overlap on

@@ -52,7 +52,7 @@ def build(force: bool = False, verbose: bool = False, jobs: int = 8) -> str:
         raise RuntimeError(f"nvcc failed for {failed}")
     tmp = LIB + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
-                           "-o", tmp, *objs, "-lcuda" if False else "-lcudart_static", "-lrt",
+                           "-o", tmp, *objs, "-lcudart_static", "-lrt",
                            "-ldl", "-lpthread"])
     os.replace(tmp, LIB)
     return LIB

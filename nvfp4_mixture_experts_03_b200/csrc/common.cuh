@@ -102,6 +102,13 @@ __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 __device__ inline void latch_status(int32_t *status, int code, int detail) {
     if (atomicCAS(&status[kStatusCode], 0, code) == 0) status[kStatusDetail] = detail;
 }
+// Detail words of NVFP4_MOE_ERR_NONFINITE when a computed value is not finite
+// (routing reports the token index instead, always < 2^20): which stored
+// intermediate, ORed with the expert id.
+enum : int { kNfH = 1 << 20, kNfY = 2 << 20, kNfOut = 3 << 20 };
+// An FP32 value stays finite when rounded to F16 iff its magnitude is below
+// 65520 (65504 plus half an F16 ulp rounds to inf); NaN fails the compare.
+__device__ inline bool fits_f16(float x) { return fabsf(x) < 65520.0f; }
 
 // --------------------------------------------------------------- utilities
 __device__ inline uint32_t smem_u32(const void *p) {

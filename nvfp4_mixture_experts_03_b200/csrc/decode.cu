@@ -363,7 +363,9 @@ __device__ inline void flush_gateup(const Params &p, const DecRoute &R, const It
                 us = atomicExch(gu + ((size_t)2 * pos + 1) * I + it.m0 + g, 0.0f);
             }
             const float gv = gs * sg * R.xsc[tok], uv = us * su * R.xsc[tok];
-            p.h[(size_t)pos * I + it.m0 + g] = __float2half_rn(silu(gv) * uv);
+            const float hf = silu(gv) * uv;
+            if (!fits_f16(hf)) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, kNfH | it.e);
+            p.h[(size_t)pos * I + it.m0 + g] = __float2half_rn(hf);
         }
     }
     __syncwarp();
@@ -383,8 +385,10 @@ __device__ inline void flush_down(const Params &p, const DecRoute &R, const Item
         const int tok = 2 * q + c;
         if (tok < p.T && R.upos[it.u * kSlots + tok] >= 0) {
             const float w = R.uw[it.u * kSlots + tok] * sd;
-            atomicAdd(p.out + (size_t)tok * p.H + it.m0 + g, acc[c] * w);
-            atomicAdd(p.out + (size_t)tok * p.H + it.m0 + g + 8, acc[2 + c] * w);
+            const float y0 = acc[c] * w, y1 = acc[2 + c] * w;
+            if (!isfinite(y0) || !isfinite(y1)) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, kNfY | it.e);
+            atomicAdd(p.out + (size_t)tok * p.H + it.m0 + g, y0);
+            atomicAdd(p.out + (size_t)tok * p.H + it.m0 + g + 8, y1);
         }
     }
 }

@@ -157,7 +157,7 @@ const char *nvfp4_moe_strerror(int s) {
         case NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
         case NVFP4_MOE_ERR_CUDA: return "CUDA error";
         case NVFP4_MOE_ERR_BAD_ROUTING: return "routing id out of range or repeated";
-        case NVFP4_MOE_ERR_NONFINITE: return "non-finite routing logit";
+        case NVFP4_MOE_ERR_NONFINITE: return "non-finite routing logit or computed value";
         case NVFP4_MOE_ERR_TIMEOUT: return "device wait timed out";
         case NVFP4_MOE_ERR_NO_DEVICE: return "no sm_100 device";
         default: return "unknown status";
@@ -429,8 +429,11 @@ __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 std::mutex g_static_mu;
 uint8_t *g_static_ptr[kMaxDevices];  // device address of g_static_scratch, per device
 
-// The array's name is only a host-side stand-in; its device address is looked up
-// once per device, with that device current.
+// Per-device set-up, once, with that device current: the array's name is only a
+// host-side stand-in, so its device address is looked up here; and the decode
+// kernels are opted into the dynamic shared memory they need (above the 48 KB
+// default at realistic layer sizes), which a process that never created a handle
+// on this device has not done yet. Neither step allocates device memory.
 int static_scratch(int dev, uint8_t **out) {
     if (dev < 0 || dev >= kMaxDevices) return NVFP4_MOE_ERR_NO_DEVICE;
     std::lock_guard<std::mutex> lock(g_static_mu);
@@ -438,6 +441,7 @@ int static_scratch(int dev, uint8_t **out) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p)
             return NVFP4_MOE_ERR_CUDA;
+        if (decode_init() != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
         g_static_ptr[dev] = static_cast<uint8_t *>(p);
     }
     *out = g_static_ptr[dev];

@@ -150,6 +150,17 @@ __device__ inline void store_half_row(uint8_t *a_stage, int r, int hf, uint4 c, 
     }
 }
 
+// Accumulator columns at or past `nvalid` belong to no pair of the tile (the MMA
+// ran over the pairs rounded up to 16, and TMEM columns past that keep whatever
+// an earlier tile left): zeroed, so that nothing computed from them is flagged
+// or stored as a real value.
+__device__ inline void zero_past(uint32_t (&v)[32], int nvalid) {
+    if (nvalid < 32) {
+#pragma unroll
+        for (int j = 0; j < 32; j++) v[j] = j < nvalid ? v[j] : 0u;
+    }
+}
+
 // Named barrier over the four epilogue warps (id 0 is __syncthreads).
 __device__ inline void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 // The same barrier with an AND over the 128 epilogue threads: every epilogue
@@ -469,6 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int il = 16 * warp + (lane & 15);
                 const bool is_gate = lane < 16;
                 const int i0 = t.m0 + kGuCta * rank;
+                bool fin = true;
 #pragma unroll 1
                 for (int c = 0; c < kChunks; c++) {
                     if (32 * c >= t.ntok) break;
@@ -485,6 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t v[32];
                     tmem_ld32(tbase + 32 * c, v);
                     tmem_ld_wait();
+                    zero_past(v, t.ntok - 32 * c);
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
                         const float mine_lo = __uint_as_float(v[j]);
@@ -494,18 +507,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float gacc = is_gate ? mine_lo : recv;
                         const float uacc = is_gate ? recv : mine_hi;
                         const float gv = gacc * sg * xs[j], uv = uacc * su * xs[j];
-                        hs[(cj0 + j) * kGuCta + il] = __float2half_rn(silu(gv) * uv);
+                        const float hf = silu(gv) * uv;
+                        fin &= fits_f16(hf);
+                        hs[(cj0 + j) * kGuCta + il] = __float2half_rn(hf);
                     }
                     epi_sync();
                     store_chunk<kGuCta>(hs, p.h + (size_t)(t.pos0 + 32 * c) * p.I + i0, p.I,
                                         min(32, t.ntok - 32 * c));
                 }
+                // h is stored in F16: a value past its range is reported, not hidden
+                if (!fin) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, kNfH | e);
             } else {
                 // y * s_d * w staged as [32 columns][128 hidden rows] F16, written into
                 // the pair's row of yp; the combine kernel sums each token's K rows in
                 // a fixed order.
                 const int r = 32 * warp + lane;
                 const int m = t.m0 + kBM * rank;
+                bool fin = true;
                 if (m < p.H) {
 #pragma unroll 1
                     for (int c = 0; c < kChunks; c++) {
@@ -522,14 +540,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint32_t v[32];
                         tmem_ld32(tbase + 32 * c, v);
                         tmem_ld_wait();
+                        zero_past(v, t.ntok - 32 * c);
 #pragma unroll
-                        for (int j = 0; j < 32; j++)
-                            ys[j * kBM + r] = __float2half_rn(__uint_as_float(v[j]) * cf[j]);
+                        for (int j = 0; j < 32; j++) {
+                            const float yf = __uint_as_float(v[j]) * cf[j];
+                            fin &= fits_f16(yf);
+                            ys[j * kBM + r] = __float2half_rn(yf);
+                        }
                         epi_sync();
                         store_chunk<kBM>(ys, p.xh + (size_t)(t.pos0 + 32 * c) * p.H + m, p.H,
                                          min(32, t.ntok - 32 * c));
                     }
                 }
+                // the per-pair rows w * s_d * y are stored in F16 (see above)
+                if (!fin) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, kNfY | e);
             }
             tc_fence_before();
             __syncwarp();

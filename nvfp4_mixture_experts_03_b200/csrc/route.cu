@@ -258,8 +258,13 @@ __global__ void __launch_bounds__(256) combine_kernel(Params p) {
                 }
             }
         }
+        bool fin = true;
 #pragma unroll
-        for (int i = 0; i < 8; i++) acc[i] += sum[i];
+        for (int i = 0; i < 8; i++) {
+            acc[i] += sum[i];
+            fin &= isfinite(acc[i]);
+        }
+        if (!fin) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, kNfOut | t);
         o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
         o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }

@@ -85,6 +85,27 @@ def test_bf16_rne_array_matches_scalar():
     assert oracle.bf16_rne_array(np.array([1.0 + 2.0 ** -8 + 2.0 ** -40]))[0] == 0x3F81
 
 
+def test_decode_matrix_equals_dense_library_decode():
+    """The oracle's whole-matrix decoder against the brute-force decoder (numpy
+    nibble split, OCP MX magnitude table, torch.float8_e4m3fn scales), element by
+    element in FP64, on random planes that include a zero group, a negative-scale
+    byte and a NaN scale byte (each must decode the same way on both sides)."""
+    g = np.random.default_rng(8)
+    rows, cols = 24, 96
+    codes = g.integers(0, 256, (rows, cols // 2), dtype=np.uint8)
+    scales = g.integers(0, 0x7F, (rows, cols // 16), dtype=np.uint8)
+    codes[3, 8:16] = 0                 # a group of zero codes (group 1 of row 3)
+    scales[5, 2] = 0                   # a zero scale
+    scales[7, 1] = 0xB8                # -1.0: a sign bit set
+    scales[9, 4] = 0x7F                # NaN
+    for glob in (1.0, 3.0517578125e-05, -0.75):
+        got = oracle.decode_matrix(codes, scales, glob)
+        ref = brute.dense(codes, scales, glob)
+        same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+        assert same.all(), (glob, np.argwhere(~same)[:4])
+    assert np.all(oracle.decode_matrix(codes, scales, 1.0)[3, 16:32] == 0.0)
+
+
 def test_dequant_products_exact_in_fp16_and_bf16():
     """code x scale has at most 6 significant bits and lies in [2^-10, 2688]: it is
     exact in both 16-bit float formats (checked exhaustively over 16 x 126 pairs)."""

@@ -3,8 +3,9 @@ intermediate 768, top-10), in the launch configuration the bench times.
 
 Weights and inputs are drawn on the GPU (synth, seeded) and copied to the host for
 the oracle. Routing (ids, counts, offsets, permutation) is compared bit for bit
-over every token; layer outputs over every token for decode, and over a spread
-sample of tokens (the oracle computes them one by one) for the long chunks."""
+over every token; layer outputs over every token for decode, and for the long
+chunks over a sample of tokens (the oracle computes them one by one) chosen so
+that every grouped-GEMM tile the kernels ran holds at least one checked pair."""
 import numpy as np
 import pytest
 import torch
@@ -18,18 +19,41 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _sample(T, ids, counts, n):
-    """n tokens: evenly spread ones plus the tokens that own the rarest used
-    experts (so cold, single-tile experts are covered)."""
-    picks = set(np.linspace(0, T - 1, n // 2).astype(int).tolist())
-    used = np.nonzero(counts)[0]
-    rare = used[np.argsort(counts[used], kind="stable")][: n]
-    for e in rare:
-        if len(picks) >= n:
-            break
-        t = int(np.nonzero((ids == e).any(axis=1))[0][0])
-        picks.add(t)
-    return np.array(sorted(picks), dtype=np.int32)
+def _sample(T, ids, counts, n, *, both_ends=True, K=None, H=2048, I=768):
+    """Tokens whose outputs are compared with the oracle: n evenly spread ones, plus
+    tokens that put a pair into every (expert, 256-pair n-tile) the grouped GEMMs
+    run -- the tile's first and last pair (both_ends), or one pair per tile at a
+    column that moves across the tile from one tile to the next. A token's output
+    depends on every row tile (gate/up: I/128 of them, down: H/256) of each n-tile
+    its pairs fall into, so the n-tiles covered times the row tiles is the number
+    of GEMM tiles checked. Returns (tokens, tiles covered, tiles run) for gate/up
+    and down."""
+    K = ids.shape[1] if K is None else K
+    picks = set(np.linspace(0, T - 1, n).astype(int).tolist())
+    # pair positions grouped by expert, then token (the layer's permutation order)
+    order = np.lexsort((np.arange(T * K), ids.reshape(-1)))
+    offs = np.concatenate([[0], np.cumsum(counts)])
+    tile_first = []
+    for e in np.nonzero(counts)[0]:
+        for i in range((int(counts[e]) + 255) // 256):
+            lo = offs[e] + 256 * i
+            hi = min(lo + 256, offs[e + 1]) - 1
+            tile_first.append((lo, hi))
+    for k, (lo, hi) in enumerate(tile_first):
+        if both_ends:
+            cols = {lo, hi}
+        else:
+            cols = {lo + (37 * k) % (hi - lo + 1)}
+        for pos in cols:
+            picks.add(int(order[pos] // K))
+    toks = np.array(sorted(picks), dtype=np.int32)
+    # tiles covered: n-tiles holding a pair of a picked token
+    mask = np.zeros(T, bool)
+    mask[toks] = True
+    covered = sum(1 for lo, hi in tile_first if mask[order[lo:hi + 1] // K].any())
+    n_tiles = len(tile_first)
+    gu_rows, dn_rows = I // 128, (H + 255) // 256
+    return toks, (covered * gu_rows, n_tiles * gu_rows), (covered * dn_rows, n_tiles * dn_rows)
 
 
 def _gpu_forward(layer_gpu, x, *, K, logits, x_scale=None, max_tokens=None):
@@ -82,7 +106,10 @@ def test_prefill_8k_full_size(big_layer):
     ref = dict(ids=ids, w=w, counts=counts, offsets=offsets, perm=perm)
     check_routing(dbg, ref, T, d.K)
     assert counts.max() > 4 * 256 and (counts == 0).any()     # skewed: multi-tile and empty experts
-    samp = _sample(T, ids, counts, 64)
+    samp, gu, dn = _sample(T, ids, counts, 64, both_ends=True, H=d.H, I=d.I)
+    print(f"8k: {len(samp)} tokens; gate/up tiles checked {gu[0]} of {gu[1]}, "
+          f"down tiles checked {dn[0]} of {dn[1]}")
+    assert gu[0] == gu[1] and dn[0] == dn[1]
     ro = oracle.moe(lg_cpu, x.cpu(), ids, w, K=d.K, sample=samp)
     assert_close(out.double().cpu().numpy()[samp], ro, "prefill 8k sample")
 
@@ -100,7 +127,10 @@ def test_w4a8_32k_full_size(big_layer):
     ids, w, _ = oracle.route(logits.cpu(), d.K)
     counts, offsets, perm = oracle.sort(ids, d.E)
     check_routing(dbg, dict(ids=ids, w=w, counts=counts, offsets=offsets, perm=perm), T, d.K)
-    samp = _sample(T, ids, counts, 48)
+    samp, gu, dn = _sample(T, ids, counts, 48, both_ends=False, H=d.H, I=d.I)
+    print(f"32k: {len(samp)} tokens; gate/up tiles checked {gu[0]} of {gu[1]}, "
+          f"down tiles checked {dn[0]} of {dn[1]}")
+    assert gu[0] == gu[1] and dn[0] == dn[1]
     ro = oracle.moe(lg_cpu, q.cpu(), ids, w, K=d.K, x_scale=qs.cpu(), sample=samp)
     assert_close(out.double().cpu().numpy()[samp], ro, "w4a8 32k sample")
 

@@ -178,3 +178,41 @@ def test_host_checks_on_device():
         m.forward(x, logits=torch.zeros(4, dims.E, device=DEV), workspace=ws)
     assert e.value.code == -4
     m.close()
+
+
+def _scaled(layer, **factors):
+    kw = {k: getattr(layer, k) for k in (
+        "gate_codes", "up_codes", "gate_scales", "up_scales", "gate_global", "up_global",
+        "down_codes", "down_scales", "down_global")}
+    for k, f in factors.items():
+        kw[k] = kw[k] * f
+    return synth.Layer(layer.dims, **kw)
+
+
+@pytest.mark.parametrize("T", [4, 64])
+@pytest.mark.parametrize("which", ["down", "gate_up"])
+def test_f16_range_overflow_is_reported_never_silent(T, which):
+    """Globals scaled by powers of two push the F16 intermediates past 65504: the
+    down global pushes the grouped-GEMM path's per-pair rows w*s_d*y out of range
+    (decode keeps y in FP32), the gate and up globals push h out of range on both
+    paths. The result must be either correct (FP32 math kept it in range) or
+    flagged NVFP4_MOE_ERR_NONFINITE -- never a silent inf in the output."""
+    dims = synth.TINY
+    base, logits, x, _ = _case(dims, T, seed=63)
+    if which == "down":
+        layer = _scaled(base, down_global=2.0 ** 24)
+    else:
+        layer = _scaled(base, gate_global=2.0 ** 10, up_global=2.0 ** 10)
+    ref = oracle.forward(layer, x, K=dims.K, logits=logits)
+    out, dbg, st = run_gpu(layer.to(DEV), x.to(DEV), K=dims.K, logits=logits.to(DEV))
+    assert np.abs(ref["out"]).max() > 65504.0 or which == "gate_up"
+    if st == 0:
+        assert_close(out, ref["out"], f"{which} scaled, T={T}")
+    else:
+        assert st == -7, st
+    if not np.all(np.isfinite(out)):
+        assert st == -7, "non-finite output without a NONFINITE status"
+    if which == "gate_up":
+        assert st == -7                 # h itself overflows F16 on both paths
+    elif T > 8:
+        assert st == -7                 # the per-pair F16 rows overflow

@@ -1,57 +1,87 @@
 """The allocation-free decode entry point, nvfp4_moe_forward_decode_static.
 
-It serves callers that cannot allocate device memory at all: they can neither
-create a handle (creation allocates a small status block) nor hand the layer a
-workspace. This test calls it through the C ABI and requires its output to match
-the regular entry point (handle + caller workspace) on the same inputs, within the
-parity tolerance, for two calls in a row: the second call reuses the library's
-static scratch, which still holds the first call's contents. It lives in a file of
-its own that pytest collects last.
+It serves callers that cannot allocate device memory at all -- code embedded in
+a runtime that owns every device allocation, or that runs where cudaMalloc is
+not allowed -- so they can neither create a handle (creation allocates a small
+status block and the decode state) nor hand the layer a workspace.
+
+The main check runs in a fresh child process, so no earlier test (and no handle)
+has touched the library on the device: the child makes two static calls in a row
+on the 512-expert, hidden 2048, intermediate 768, top-10 layer (8 tokens, then
+1 token; the second call reuses the static scratch, which still holds the first
+call's contents) before any handle exists, then creates a regular handle and
+requires both static outputs to match the regular entry point (handle + caller
+workspace) and the FP64 oracle within the parity tolerance. It lives in a file
+of its own that pytest collects last.
 """
-import ctypes as C
+import os
+import subprocess
+import sys
 
-import numpy as np
 import pytest
-import torch
 
-import synth
-from helpers import assert_close
-
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 pytestmark = pytest.mark.gpu
 
-DEV = "cuda"
 
+def _child():
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import torch
 
-def _io(nv, x, logits, out):
-    return nv.IO(x.shape[0], nv.ACT_BF16, x.data_ptr(), None, logits.data_ptr(), None, None,
-                 nv.OUT_F32, out.data_ptr(), None, None, None, None, None)
-
-
-def test_static_decode_matches_regular_entry_point_twice():
     import nvfp4_mixture_experts_03_b200 as nv
-    dims = synth.LayerDims(E=64, H=512, I=384, K=6)
-    layer = synth.make_layer(dims, seed=901).to(DEV)
-    regular = nv.MoELayer.from_layer(layer, top_k=dims.K, max_tokens=8)
-    cd = nv.Dims(dims.H, dims.I, dims.E, dims.K, 8)
+    import oracle
+    import synth
+    from helpers import assert_close
+
+    wl = synth.CONFIGS["decode"]
+    d = wl.dims
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    layer = synth.make_layer(d, synth.workload_seed(wl, 5), device=dev)
+    cd = nv.Dims(d.H, d.I, d.E, d.K, nv.DECODE_MAX_T)
     cw = nv.Weights(*[t.data_ptr() for t in layer.planes()])
     stream = torch.cuda.current_stream().cuda_stream
-    for call, T in enumerate((8, 3)):
-        x = synth.make_x_bf16(T, dims.H, seed=910 + call, outliers=True, device=DEV)
-        logits = synth.make_logits(T, dims.E, seed=920 + call, zipf_s=1.1, device=DEV)
+    calls = []
+    for call, T in enumerate((8, 1)):
+        seed = synth.workload_seed(wl, 5) + 100 + call
+        x = synth.make_x_bf16(T, d.H, seed, outliers=True, device=dev)
+        logits = synth.make_logits(T, d.E, seed, zipf_s=wl.zipf_s, device=dev)
+        got = torch.full((T, d.H), float("nan"), dtype=torch.float32, device=dev)
+        io = nv.IO(T, nv.ACT_BF16, x.data_ptr(), None, logits.data_ptr(), None, None,
+                   nv.OUT_F32, got.data_ptr(), None, None, None, None, None)
+        rc = nv.nvfp4_moe_forward_decode_static(cd, cw, io, stream)
+        assert rc == 0, f"static call {call + 1}: {nv.nvfp4_moe_strerror(rc)}"
+        calls.append((x, logits, got))
+    torch.cuda.synchronize()
+    # only now a regular handle: the static calls above ran without one
+    regular = nv.MoELayer.from_layer(layer, top_k=d.K, max_tokens=nv.DECODE_MAX_T)
+    lc = layer.to("cpu")
+    for call, (x, logits, got) in enumerate(calls):
         want = regular.forward(x, logits=logits)
-        got = torch.full((T, dims.H), float("nan"), dtype=torch.float32, device=DEV)
-        rc = nv.nvfp4_moe_forward_decode_static(cd, cw, _io(nv, x, logits, got), stream)
-        assert rc == 0, nv.nvfp4_moe_strerror(rc)
-        torch.cuda.synchronize()
-        assert_close(got.double().cpu().numpy(), want.double().cpu().numpy(),
-                     f"static decode call {call + 1}")
+        assert regular.status() == 0
+        g = got.double().cpu().numpy()
+        assert_close(g, want.double().cpu().numpy(), f"static vs regular, call {call + 1}")
+        ref = oracle.forward(lc, x.cpu(), K=d.K, logits=logits.cpu())["out"]
+        l2, mr = assert_close(g, ref, f"static vs oracle, call {call + 1}")
+        print(f"call {call + 1} (T={x.shape[0]}): vs oracle l2 {l2:.2e} maxrel {mr:.2e}")
     regular.close()
+    print("CHILD_OK")
+
+
+def test_static_decode_in_fresh_process_matches_regular_and_oracle():
+    r = subprocess.run([sys.executable, os.path.abspath(__file__), "--child"], cwd=ROOT,
+                       capture_output=True, text=True, timeout=600)
+    print(r.stdout[-2000:])
+    assert r.returncode == 0 and "CHILD_OK" in r.stdout, r.stdout[-3000:] + r.stderr[-3000:]
 
 
 def test_static_decode_rejects_sizes_beyond_its_scratch():
+    import torch
+
     import nvfp4_mixture_experts_03_b200 as nv
     fake = nv.Weights(*[(1 << 40) + i * (1 << 30) for i in range(9)])
-    x = torch.zeros(1, dtype=torch.uint8, device=DEV)
+    x = torch.zeros(1, dtype=torch.uint8, device="cuda")
     big = nv.Dims(8192, 8192, 64, 16, 8)          # h alone needs 8*16*8192*2 B = 2 MiB
     io = nv.IO(8, nv.ACT_BF16, x.data_ptr(), None, x.data_ptr(), None, None, nv.OUT_F32,
                x.data_ptr(), None, None, None, None, None)
@@ -59,3 +89,7 @@ def test_static_decode_rejects_sizes_beyond_its_scratch():
     small = nv.Dims(256, 128, 8, 2, 16)
     io.T = 9                                          # beyond the decode path
     assert nv.nvfp4_moe_forward_decode_static(small, fake, io, 0) == -2
+
+
+if __name__ == "__main__" and "--child" in sys.argv:
+    _child()
