@@ -44,9 +44,8 @@
  *     owned by the caller. The handle BORROWS the weight pointers: they must stay
  *     valid until nvfp4_moe_destroy. The library allocates no device memory
  *     except what nvfp4_moe_create makes: a 256-byte status block and, when
- *     max_tokens >= 1, the decode state (a few counters plus FP32 partial sums
- *     of min(max_tokens, 8) * top_k token slots x 2 x inter: 0.5 MB for the
- *     512-expert, 2048/768, top-10 layer), kept zero between calls.
+ *     the layer can take the decode kernel, its state (2304 bytes of counters),
+ *     kept zero between calls.
  *   - All other scratch lives in the caller's workspace (nvfp4_moe_workspace_bytes).
  *
  * Errors: every call returns 0 (NVFP4_MOE_OK) or a negative nvfp4_moe_status.
@@ -68,10 +67,15 @@
  *   upstream Strata": folding a tiny scale into FP16 activations pushed them
  *   into FP16 subnormals).
  *
- * Co-residency: the decode kernel (T <= 8) runs one CTA per SM and its CTAs wait
- *   on one another through counters (bounded). It assumes the GPU is not shared
- *   with other work that keeps SMs busy for long; otherwise such waits can run
- *   out and the call reports NVFP4_MOE_ERR_TIMEOUT.
+ * Decode: calls with T <= 8 run one decode kernel (one CTA per SM) when
+ *   H <= 6144 and I <= 6144 (its shared-memory rings must hold at least two items
+ *   of each projection: 9 * H and 9 * I bytes each); other layers run small
+ *   batches through the grouped-GEMM path. The decode kernel adds each token's
+ *   K expert rows in the fixed order j = 0..K-1 and uses no floating-point
+ *   atomics, so, like the grouped-GEMM path, it returns the same bits on every
+ *   run. Its CTAs wait on one another through counters (bounded). It assumes the
+ *   GPU is not shared with other work that keeps SMs busy for long; otherwise
+ *   such waits can run out and the call reports NVFP4_MOE_ERR_TIMEOUT.
  *
  * Threading: a handle may be used from one host thread at a time. Two forward
  *   calls that run concurrently on the GPU must not share a workspace.
@@ -103,7 +107,7 @@ extern "C" {
 typedef enum {
     NVFP4_MOE_OK = 0,
     NVFP4_MOE_ERR_INVALID_ARG = -1,        /* null pointer, T<0, T>max_tokens, bad enum   */
-    NVFP4_MOE_ERR_UNSUPPORTED_DIMS = -2,   /* H or I not a multiple of 128; K>E; K>16; E>1024;
+    NVFP4_MOE_ERR_UNSUPPORTED_DIMS = -2,   /* H or I not a multiple of 32; K>E; K>16; E>1024;
                                               max_tokens > 65536                              */
     NVFP4_MOE_ERR_MISALIGNED = -3,         /* a plane or buffer not 16-byte aligned       */
     NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL = -4,
@@ -119,7 +123,10 @@ typedef enum {
 typedef struct nvfp4_moe nvfp4_moe_t; /* opaque handle */
 
 /* Layer geometry. hidden = H, inter = I, n_experts = E, top_k = K.
- * max_tokens bounds T for every forward call and sizes the workspace. */
+ * max_tokens bounds T for every forward call and sizes the workspace.
+ * H and I must be multiples of 32: whole groups of 16 inputs per scale ("TensorFold
+ * PR #906", first post: cuts keep groups of 16) and code rows of a multiple of 16
+ * bytes, which the tensor-map copies need. */
 typedef struct {
     int32_t hidden;
     int32_t inter;
@@ -250,10 +257,12 @@ NVFP4_MOE_API int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events
  * __device__ array: every GPU that loads the library holds it until the process
  * exits). dims and weights are checked exactly as by nvfp4_moe_create; io and
  * stream are as for nvfp4_moe_forward. Calls no cudaMalloc/cudaFree.
- *   - T > 8 returns NVFP4_MOE_ERR_UNSUPPORTED_DIMS; a layer whose decode
- *     scratch and state for this T exceed 2 MiB - 256 bytes returns
- *     NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL (e.g. H = I = 8192 with K = 16). Both
- *     are checked before anything is enqueued. T = 0 is a no-op.
+ *   - T > 8, or a layer outside the decode kernel (see "Decode" above),
+ *     returns NVFP4_MOE_ERR_UNSUPPORTED_DIMS; a layer whose decode scratch and
+ *     state for this T exceed 2 MiB - 256 bytes returns
+ *     NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL (e.g. H = I = 4096 with K = 16 at
+ *     T = 8: the FP32 per-pair down rows alone take 2 MiB). Both are checked
+ *     before anything is enqueued. T = 0 is a no-op.
  *   - The first call on a device does a one-time set-up there: it looks up the
  *     array's device address (cudaGetSymbolAddress) and opts the decode kernels
  *     into the shared memory they need (cudaFuncSetAttribute). Make that first

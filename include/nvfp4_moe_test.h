@@ -26,6 +26,14 @@ extern "C" {
  * NVFP4_MOE_ERR_INVALID_ARG for a NULL handle or an unknown flag. */
 NVFP4_MOE_API int nvfp4_moe_test_set_flags(nvfp4_moe_t *h, int32_t flags);
 
+/* The detail word that came with the status the last nvfp4_moe_get_status on h
+ * returned (0 when it returned 0). For NVFP4_MOE_ERR_NONFINITE raised by a
+ * computed value: (1 << 20) | expert for h, (2 << 20) | expert for a per-pair
+ * down row, (3 << 20) | (token or first row) for the output; a token index for a
+ * routing logit. For NVFP4_MOE_ERR_TIMEOUT: where the wait gave up. Returns 0 for
+ * a NULL handle. */
+NVFP4_MOE_API int nvfp4_moe_test_last_detail(const nvfp4_moe_t *h);
+
 /* Makes the n-th device allocation (counting from 1) made by later
  * nvfp4_moe_create calls fail as if the device were out of memory; the hook
  * then disarms itself. n <= 0 disarms it. create must then return

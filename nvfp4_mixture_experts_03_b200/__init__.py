@@ -32,7 +32,7 @@ EXPORTS = ("nvfp4_moe_create", "nvfp4_moe_workspace_bytes", "nvfp4_moe_forward",
            "nvfp4_moe_get_status", "nvfp4_moe_destroy", "nvfp4_moe_strerror",
            "nvfp4_moe_abi_version", "nvfp4_moe_set_phase_events",
            "nvfp4_moe_forward_decode_static",
-           "nvfp4_moe_test_set_flags", "nvfp4_moe_test_fail_alloc")
+           "nvfp4_moe_test_set_flags", "nvfp4_moe_test_fail_alloc", "nvfp4_moe_test_last_detail")
 TEST_DECODE_STALL = 1   # include/nvfp4_moe_test.h
 PHASE_EVENTS = 5
 
@@ -90,6 +90,8 @@ def lib() -> C.CDLL:
         L.nvfp4_moe_abi_version.restype = C.c_int
         L.nvfp4_moe_set_phase_events.restype = C.c_int
         L.nvfp4_moe_set_phase_events.argtypes = [C.c_void_p, C.POINTER(C.c_void_p), C.c_int32]
+        L.nvfp4_moe_test_last_detail.restype = C.c_int
+        L.nvfp4_moe_test_last_detail.argtypes = [C.c_void_p]
         L.nvfp4_moe_forward_decode_static.restype = C.c_int
         L.nvfp4_moe_forward_decode_static.argtypes = [C.POINTER(Dims), C.POINTER(Weights),
                                                       C.POINTER(IO), C.c_void_p]
@@ -145,6 +147,11 @@ def nvfp4_moe_test_set_flags(handle: int, flags: int) -> int:
     """Test hook (include/nvfp4_moe_test.h): TEST_DECODE_STALL makes decode's bounded
     waits run out, so the call latches TIMEOUT."""
     return lib().nvfp4_moe_test_set_flags(C.c_void_p(handle), C.c_int32(flags))
+
+
+def nvfp4_moe_test_last_detail(handle: int) -> int:
+    """Test hook: the detail word of the status the last get_status returned."""
+    return lib().nvfp4_moe_test_last_detail(C.c_void_p(handle))
 
 
 def nvfp4_moe_test_fail_alloc(n: int) -> None:

@@ -25,18 +25,15 @@ constexpr int kGuRows = 128;           // intermediates per gate/up tile (64 per
 constexpr int kDnRows = 256;           // hidden rows per down tile (128 per CTA; the last may be half)
 
 // Device status block layout (int32 words, 256 bytes): the latched error and its
-// detail, and the decode kernel's grid-wide barrier (generation word, top-level
-// arrival count, kBarGroups group arrival counts).
-enum : int { kStatusCode = 0, kStatusDetail = 1, kStatusBarGen = 8, kStatusBarTop = 9,
-             kStatusBarGroup = 16, kBarGroups = 16, kStatusWords = 64 };
+// detail.
+enum : int { kStatusCode = 0, kStatusDetail = 1, kStatusWords = 64 };
 
 // Per-call routing/tile counters kept in the workspace (int32 words).
 enum : int { kCntTilesGu = 0, kCntTilesDn = 1, kCntUniq = 2, kCntWords = 64 };
-// Decode state (per handle, zero between launches): int words, then the FP32
-// gate/up partial sums [pairs][2][I]. kDsStaged: CTAs past their activation
-// reads; kDsExit: CTAs done; kDsReady + u: finished gate/up items of used
-// expert u; kDsItems + item: K rounds summed so far of a split gate/up item.
-enum : int { kDsStaged = 0, kDsExit = 1, kDsReady = 2, kDsItems = 2 + 128 };
+// Decode state (per handle, int32 words, zero between launches). kDsDone: CTAs
+// whose down rows are written; kDsExit: CTAs done; kDsReady + u: finished gate/up
+// items of used expert u (u < 128).
+enum : int { kDsDone = 0, kDsExit = 1, kDsReady = 2, kDsWords = 2 + 128 };
 
 struct Tile {  // one grouped-GEMM tile
     int32_t expert;   // expert id
@@ -75,9 +72,10 @@ struct Params {
     float *pw;                 // [P] routing weight at each position
     float *ps;                 // [P] activation scale at each position (prefill)
     float *xscale;             // [T] activation scale per token
+    float *ph;                 // [P] prefill: 2^hexp of the pair's token at each position
+    float *phinv;              // [T] prefill: 2^-hexp per token
     Tile *tiles_gu, *tiles_dn;
-    int32_t *uniq;             // [<=P] decode: unique experts ascending
-    int32_t *upos;             // [<=P][8] decode: position of (unique expert, token) or -1
+    float *ybuf;               // decode: [P][H] FP32 w * s_d * y per pair position
     __half *xh;                // prefill: [P][H] F16 activations per pair position, then the
                                // down projection's w * s_d * y per pair (F16)
     __half *h;                 // [P][I]
@@ -89,8 +87,7 @@ struct Params {
     int32_t nch;               // routing chunks
     int32_t max_tiles_gu, max_tiles_dn;
     int32_t *dstate;           // decode: counters (kDs*), zero between launches
-    float *dgu;                // decode: [pairs][2][I] FP32 partial sums, zero between launches
-    int32_t dec_hs_rows;       // decode: h rows one CTA stages for its down range
+    int32_t dec_n1, dec_n2;    // decode: ring slots for gate/up and for down items
     int32_t test_flags;        // NVFP4_MOE_TEST_* (test hooks; 0 in production)
 };
 
@@ -379,20 +376,30 @@ __device__ inline int pow2_shift_for(float amax) {
     return k < -120 ? -120 : (k > 120 ? 120 : k);   // keep 2^-k a normal FP32
 }
 
+// Power-of-two exponent by which a token's h values are stored (h * 2^e; also
+// the grouped-GEMM path's per-pair down rows, which are built from h): 0 while
+// the token's activation amax stays below 256, else -2 (m - 8) for an amax in
+// [2^(m-1), 2^m), so that h, which grows with the square of the activations,
+// keeps within F16's range. Exact (a power of two), undone in FP32.
+__device__ inline int h_exp_for(float amax) {
+    if (!(amax >= 256.0f) || !isfinite(amax)) return 0;
+    int m;
+    frexpf(amax, &m);           // amax in [2^(m-1), 2^m), m >= 9
+    const int e = -2 * (m - 8);
+    return e < -100 ? -100 : e;
+}
+
 // ------------------------------------------------------------ kernel decls
 void launch_route_large(const Params &p, cudaStream_t s);
 void launch_prep_prefill(const Params &p, cudaStream_t s);
 void launch_combine(const Params &p, cudaStream_t s);   // prefill: per-token sum of the K pair rows
 cudaError_t launch_decode(const Params &p, cudaStream_t s);   // the whole T <= 8 layer
 int decode_grid();                                 // CTAs of the decode kernel (one per SM)
-int decode_hs_rows(int T, int K, int E, int grid); // h rows one decode CTA may stage
-// Bytes of the decode state for up to `pairs` (token, slot) pairs.
-inline size_t decode_state_ints_bytes(int pairs, int inter) {
-    return (((size_t)kDsItems + (size_t)pairs * (inter / 8)) * 4 + 255) & ~size_t(255);
-}
-inline size_t decode_state_bytes(int pairs, int inter) {
-    return decode_state_ints_bytes(pairs, inter) + (size_t)pairs * 2 * inter * 4;
-}
+// Whether the decode kernel's shared-memory plan holds layers of these dims (else
+// small batches take the grouped-GEMM path).
+bool decode_fits(int H, int I);
+// Bytes of the decode state (kDsWords counters).
+inline size_t decode_state_bytes() { return ((size_t)kDsWords * 4 + 255) & ~size_t(255); }
 // mode 0: gate/up + SwiGLU, map_b = F16 activations [P][H]; mode 1: down, map_b =
 // h [P][I]; both 64 x 64 boxes
 // Tensor maps of the packed E2M1 code planes (bytes; 128-byte x 64-row boxes for

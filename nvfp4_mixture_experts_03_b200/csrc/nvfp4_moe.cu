@@ -26,10 +26,10 @@ struct nvfp4_moe {
     int pf_clusters;  // resident CTA pairs of the prefill GEMMs
     CodeMaps codes;   // tensor maps of the weight code planes (prefill GEMMs)
     int32_t *status;  // kStatusWords ints on the device
-    uint8_t *dstate;  // decode state (zero between launches), for dec_pairs pairs
+    uint8_t *dstate;  // decode state (counters, zero between launches), or null
     size_t dstate_bytes;
-    int dec_pairs;
     int32_t test_flags;  // NVFP4_MOE_TEST_* (test hooks)
+    int32_t last_detail; // detail word of the status the last get_status returned
     cudaEvent_t phase[NVFP4_MOE_PHASE_EVENTS];
     bool phase_on;
 };
@@ -98,9 +98,14 @@ cudaError_t dev_alloc(void **p, size_t bytes) {
 inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 inline bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
 
+// Whether a call with T tokens takes the decode kernel (else the grouped GEMMs).
+bool use_decode(const nvfp4_moe_dims &d, int T) {
+    return T <= NVFP4_MOE_DECODE_MAX_T && decode_fits(d.hidden, d.inter);
+}
+
 struct WsLayout {
-    size_t cnt, ids, wts, hist, cbase, counts, offsets, perm, inv, ptok, pw, ps, xscale, tiles_gu,
-        tiles_dn, uniq, upos, xh, h, total;
+    size_t cnt, ids, wts, hist, cbase, counts, offsets, perm, inv, ptok, pw, ps, xscale, ph, phinv, tiles_gu,
+        tiles_dn, ybuf, xh, h, total;
     int nch, max_gu, max_dn;
 };
 
@@ -109,9 +114,9 @@ WsLayout layout(const nvfp4_moe_dims &d, int T) {
     const size_t P = (size_t)T * d.top_k;
     const int E = d.n_experts;
     L.nch = cdiv(T > 0 ? T : 1, kChunkTokens);
-    const bool decode = T <= NVFP4_MOE_DECODE_MAX_T;
+    const bool decode = use_decode(d, T);
     const size_t ntile_n = P / kBN + (size_t)(E < (int)P ? E : (int)P) + 1;
-    L.max_gu = decode ? 0 : (int)(ntile_n * (d.inter / kGuRows));
+    L.max_gu = decode ? 0 : (int)(ntile_n * cdiv(d.inter, kGuRows));
     L.max_dn = decode ? 0 : (int)(ntile_n * cdiv(d.hidden, kDnRows));
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -132,10 +137,11 @@ WsLayout layout(const nvfp4_moe_dims &d, int T) {
     L.pw = take(P * 4);
     L.ps = take(P * 4);
     L.xscale = take((size_t)T * 4);
+    L.ph = take(decode ? 0 : P * 4);
+    L.phinv = take(decode ? 0 : (size_t)T * 4);
     L.tiles_gu = take((size_t)L.max_gu * sizeof(Tile));
     L.tiles_dn = take((size_t)L.max_dn * sizeof(Tile));
-    L.uniq = take(decode ? P * 4 : 0);
-    L.upos = take(decode ? P * NVFP4_MOE_DECODE_MAX_T * 4 : 0);
+    L.ybuf = take(decode ? P * d.hidden * 4 : 0);   // decode: FP32 down rows per pair
     L.xh = take(decode ? 0 : P * d.hidden * 2);   // decode stages activations in shared memory
     L.h = take(P * d.inter * 2);
     L.total = o;
@@ -172,7 +178,7 @@ int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
     const nvfp4_moe_dims d = *dims;
     if (d.hidden <= 0 || d.inter <= 0 || d.n_experts <= 0 || d.top_k <= 0 || d.max_tokens < 0)
         return NVFP4_MOE_ERR_INVALID_ARG;
-    if (d.hidden % 128 || d.inter % 128 || d.top_k > d.n_experts ||
+    if (d.hidden % 32 || d.inter % 32 || d.top_k > d.n_experts ||
         d.top_k > NVFP4_MOE_MAX_TOPK || d.n_experts > 1024)
         return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
     if (d.max_tokens > NVFP4_MOE_MAX_TOKENS) return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
@@ -214,9 +220,8 @@ int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
     h->dstate = nullptr;
     h->phase_on = false;
     h->test_flags = 0;
-    const int dec_t = d.max_tokens < NVFP4_MOE_DECODE_MAX_T ? d.max_tokens : NVFP4_MOE_DECODE_MAX_T;
-    h->dec_pairs = dec_t * d.top_k;
-    h->dstate_bytes = h->dec_pairs > 0 ? decode_state_bytes(h->dec_pairs, d.inter) : 0;
+    h->last_detail = 0;
+    h->dstate_bytes = d.max_tokens >= 1 && use_decode(d, 1) ? decode_state_bytes() : 0;
     if (dev_alloc(reinterpret_cast<void **>(&h->status), kStatusWords * sizeof(int32_t)) != cudaSuccess ||
         cudaMemset(h->status, 0, kStatusWords * sizeof(int32_t)) != cudaSuccess ||
         (h->dstate_bytes &&
@@ -297,10 +302,11 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     p.pw = reinterpret_cast<float *>(b + L.pw);
     p.ps = reinterpret_cast<float *>(b + L.ps);
     p.xscale = reinterpret_cast<float *>(b + L.xscale);
+    p.ph = reinterpret_cast<float *>(b + L.ph);
+    p.phinv = reinterpret_cast<float *>(b + L.phinv);
     p.tiles_gu = reinterpret_cast<Tile *>(b + L.tiles_gu);
     p.tiles_dn = reinterpret_cast<Tile *>(b + L.tiles_dn);
-    p.uniq = reinterpret_cast<int32_t *>(b + L.uniq);
-    p.upos = reinterpret_cast<int32_t *>(b + L.upos);
+    p.ybuf = reinterpret_cast<float *>(b + L.ybuf);
     p.xh = reinterpret_cast<__half *>(b + L.xh);
     p.h = reinterpret_cast<__half *>(b + L.h);
     p.status = h->status;
@@ -313,11 +319,10 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     p.max_tiles_gu = L.max_gu;
     p.max_tiles_dn = L.max_dn;
     p.test_flags = h->test_flags;
-    if (T <= NVFP4_MOE_DECODE_MAX_T) {
-        if (T * d.top_k > h->dec_pairs || !h->dstate) return NVFP4_MOE_ERR_INVALID_ARG;
+    const bool decode = use_decode(d, T);
+    if (decode) {
+        if (!h->dstate) return NVFP4_MOE_ERR_INVALID_ARG;
         p.dstate = reinterpret_cast<int32_t *>(h->dstate);
-        p.dgu = reinterpret_cast<float *>(h->dstate + decode_state_ints_bytes(h->dec_pairs, d.inter));
-        p.dec_hs_rows = decode_hs_rows(T, d.top_k, d.n_experts, decode_grid());
     }
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -333,7 +338,7 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
         else
             cudaEventRecord(h->phase[i], s);
     };
-    if (T <= NVFP4_MOE_DECODE_MAX_T) {
+    if (decode) {
         // one kernel for the whole decode layer: its routing, staging and both
         // projections are not separable by events (phases 0-2 and 3-4 coincide)
         mark(0);
@@ -371,7 +376,8 @@ int nvfp4_moe_get_status(nvfp4_moe_t *h, void *stream) {
     if (cudaMemcpy(st, h->status, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
         return NVFP4_MOE_ERR_CUDA;
     if (cudaMemset(h->status, 0, sizeof(st)) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
-    // A launch that gave up may have left decode counts or partial sums behind.
+    h->last_detail = st[kStatusCode] != 0 ? st[kStatusDetail] : 0;
+    // A launch that gave up may have left decode counts behind.
     if (st[kStatusCode] != 0 && h->dstate && cudaMemset(h->dstate, 0, h->dstate_bytes) != cudaSuccess)
         return NVFP4_MOE_ERR_CUDA;
     return st[kStatusCode];
@@ -396,6 +402,8 @@ int nvfp4_moe_test_set_flags(nvfp4_moe_t *h, int32_t flags) {
     h->test_flags = flags;
     return NVFP4_MOE_OK;
 }
+
+int nvfp4_moe_test_last_detail(const nvfp4_moe_t *h) { return h ? h->last_detail : 0; }
 
 void nvfp4_moe_test_fail_alloc(int32_t n) { g_fail_alloc = n > 0 ? n : 0; }
 
@@ -454,7 +462,7 @@ int check_layer(const nvfp4_moe_dims *dims, const nvfp4_moe_weights *w) {
     const nvfp4_moe_dims d = *dims;
     if (d.hidden <= 0 || d.inter <= 0 || d.n_experts <= 0 || d.top_k <= 0 || d.max_tokens < 0)
         return NVFP4_MOE_ERR_INVALID_ARG;
-    if (d.hidden % 128 || d.inter % 128 || d.top_k > d.n_experts ||
+    if (d.hidden % 32 || d.inter % 32 || d.top_k > d.n_experts ||
         d.top_k > NVFP4_MOE_MAX_TOPK || d.n_experts > 1024 || d.max_tokens > NVFP4_MOE_MAX_TOKENS)
         return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
     const void *planes[] = {w->gate_codes, w->up_codes, w->gate_scales, w->up_scales,
@@ -481,10 +489,9 @@ int nvfp4_moe_forward_decode_static(const nvfp4_moe_dims *dims, const nvfp4_moe_
     if (rc != NVFP4_MOE_OK) return rc;
     if (!io) return NVFP4_MOE_ERR_INVALID_ARG;
     if (io->T < 0 || io->T > dims->max_tokens) return NVFP4_MOE_ERR_INVALID_ARG;
-    if (io->T > NVFP4_MOE_DECODE_MAX_T) return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
+    if (io->T > NVFP4_MOE_DECODE_MAX_T || !use_decode(*dims, io->T)) return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
     if (io->T == 0) return NVFP4_MOE_OK;
-    const int pairs = io->T * dims->top_k;
-    const size_t state = decode_state_bytes(pairs, dims->inter);
+    const size_t state = decode_state_bytes();
     const size_t need = layout(*dims, io->T).total;
     if (need + state > kStaticScratchBytes - kStaticStatusBytes) return NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL;
     int dev = 0;
@@ -503,21 +510,20 @@ int nvfp4_moe_forward_decode_static(const nvfp4_moe_dims *dims, const nvfp4_moe_
     h.w = *w;
     h.device = dev;
     h.num_sms = sms;
-    h.pf_clusters = 0;   // T <= 8 never reaches the prefill GEMMs
+    h.pf_clusters = 0;   // the decode kernel never reaches the prefill GEMMs
     h.test_flags = 0;
+    h.last_detail = 0;
     h.status = reinterpret_cast<int32_t *>(scratch);
     h.dstate = scratch + kStaticStatusBytes;
     h.dstate_bytes = state;
-    h.dec_pairs = pairs;
     h.phase_on = false;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // The status words and the decode state must start at zero (the status
+    // The status words and the decode counters must start at zero (the status
     // latches the first device error; an earlier call that gave up may have left
-    // decode counts behind, and no status read follows a call here).
+    // counts behind, and no status read follows a call here).
     if (cudaMemsetAsync(scratch, 0, kStaticStatusBytes + state, s) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
     return nvfp4_moe_forward(&h, io, scratch + kStaticStatusBytes + state,
                              kStaticScratchBytes - kStaticStatusBytes - state, stream);
 }
 
 }  // extern "C"
-

@@ -58,7 +58,7 @@ constexpr int kRawBytes = kRawCodeBytes + kRawScaleBytes;
 static_assert(kRing % 2 == 0 && kRawSteps % 2 == 0, "the dequant warps fill ring stages in pairs");
 constexpr int kTmemCols = 512;                 // two 256-column accumulators
 constexpr int kEpiBytes = 2 * 32 * kBM * 2;    // epilogue staging: 2 x (32 columns x 128 rows x F16)
-constexpr int kColBytes = kBN * 4;            // the tile's per-column factors (FP32)
+constexpr int kColBytes = kBN * 4;            // one per-column factor array of a tile (FP32)
 constexpr uint64_t kDrainNs = 200000000ull;    // bounded drain on abort
 constexpr uint64_t kSettleNs = 1000000ull;     // lets in-flight copies land after an abort
 constexpr uint16_t kBothCtas = 0x3;
@@ -77,7 +77,7 @@ struct __align__(8) Bars {
 };
 
 constexpr size_t smem_bytes() {
-    return 1024 + kRing * (kAStage + kBStage) + kRawStages * kRawBytes + kEpiBytes + kColBytes +
+    return 1024 + kRing * (kAStage + kBStage) + kRawStages * kRawBytes + kEpiBytes + 2 * kColBytes +
            sizeof(Bars);
 }
 
@@ -178,13 +178,14 @@ __device__ inline bool epi_all(bool v) {
 
 // Copies a staged chunk (ncol columns of kRowsB F16 values, each column contiguous
 // in shared memory) to `ncol` rows of `dst` (row stride `ld` elements), by the 128
-// epilogue threads with 16-byte accesses. Every shared load is issued before the
+// epilogue threads with 16-byte accesses; only the first `nrows` values of each
+// column (a multiple of 8) are stored. Every shared load is issued before the
 // first global store: the compiler cannot tell the two apart and would otherwise
 // wait for each store before the next load.
 template <int kRowsB>
-__device__ inline void store_chunk(const __half *stage, __half *dst, size_t ld, int ncol) {
+__device__ inline void store_chunk(const __half *stage, __half *dst, size_t ld, int ncol, int nrows) {
     constexpr int kParts = kRowsB / 8, kPer = 32 * kParts / 128;
-    const int nq = ncol * kParts;
+    const int nq = ncol * kParts, vparts = nrows / 8;
     uint4 val[kPer];
 #pragma unroll
     for (int k = 0; k < kPer; k++) {
@@ -194,7 +195,8 @@ __device__ inline void store_chunk(const __half *stage, __half *dst, size_t ld, 
 #pragma unroll
     for (int k = 0; k < kPer; k++) {
         const int q = threadIdx.x + 128 * k;
-        if (q < nq) reinterpret_cast<uint4 *>(dst + (size_t)(q / kParts) * ld)[q % kParts] = val[k];
+        if (q < nq && q % kParts < vparts)
+            reinterpret_cast<uint4 *>(dst + (size_t)(q / kParts) * ld)[q % kParts] = val[k];
     }
 }
 
@@ -211,7 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *raw_base = b_base + kRing * kBStage;
     uint8_t *epi_stage = raw_base + kRawStages * kRawBytes;
     float *colf_s = reinterpret_cast<float *>(epi_stage + kEpiBytes);
-    Bars *bars = reinterpret_cast<Bars *>(epi_stage + kEpiBytes + kColBytes);
+    float *colu_s = colf_s + kBN;                 // gate/up: the up factor (see the epilogue)
+    Bars *bars = reinterpret_cast<Bars *>(epi_stage + kEpiBytes + 2 * kColBytes);
     volatile int *abort = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -221,7 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const Tile *tiles = MODE == 0 ? p.tiles_gu : p.tiles_dn;
     const int ntiles = p.cnt[MODE == 0 ? kCntTilesGu : kCntTilesDn];
     const int Kdim = MODE == 0 ? p.H : p.I;
-    const int nk = Kdim / kBK;
+    // K steps: K rounded up to a multiple of 128 (the dequant warps take steps in
+    // pairs); codes past K arrive as zeros (tensor-map fill) and their scales are
+    // written as zeros, so the padding adds nothing.
+    const int nk = 2 * cdiv(Kdim, 2 * kBK);
     const int ntl = ntiles > cid ? cdiv(ntiles - cid, ncl) : 0;
 
     if (threadIdx.x == 0) {
@@ -315,8 +321,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Per tile and 4 K steps: the codes of this CTA's 128 rows by TMA (one
         // 64-row box per gate and up plane, or one 128-row box of down), the
         // scales by 8-byte copies from all 32 lanes (a scale row's stride need
-        // not be a multiple of 16 bytes, which a tensor map would require).
+        // not be a multiple of 16 bytes, which a tensor map would require). When K
+        // is not a multiple of 128 a row's scales need not be 8-byte aligned: they
+        // are then copied 2 bytes at a time by plain loads, with zeros past the
+        // row's end and for rows past the plane (a partial last tile of the last
+        // expert).
         const int kd16 = Kdim / 16;   // scale bytes per weight row
+        const bool narrow = Kdim % 128 != 0;
+        const int plane_rows = MODE == 0 ? p.E * p.I : p.E * p.H;
         Ring<kRawStages> rr;
         uint32_t issued = 0, issued_phase = 0;
         bool ok = true;
@@ -343,18 +355,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                     issued |= 1u << rr.stage;
                     issued_phase = (issued_phase & ~(1u << rr.stage)) | (rr.phase << rr.stage);
                 }
-                // 128 rows x two 8-byte pieces; pieces past the row's end are skipped
+                if (!narrow) {
+                    // 128 rows x two 8-byte pieces; pieces past the row's end are
+                    // skipped (their K steps are never converted), and so are rows
+                    // past the plane (their codes arrive as zeros and their results
+                    // are dropped)
 #pragma unroll
-                for (int k = 0; k < (2 * kBM) / 32; k++) {
-                    const int ci = lane + 32 * k, row = ci >> 1, off = 16 * R + 8 * (ci & 1);
-                    if (off < kd16) {
-                        const uint8_t *src = MODE == 0 ? (row < 64 ? sc0 + (size_t)row * kd16
-                                                                   : sc1 + (size_t)(row - 64) * kd16)
-                                                       : sc0 + (size_t)row * kd16;
-                        cp_async8(raw + kRawCodeBytes + row * 16 + 8 * (ci & 1), src + off);
+                    for (int k = 0; k < (2 * kBM) / 32; k++) {
+                        const int ci = lane + 32 * k, row = ci >> 1, off = 16 * R + 8 * (ci & 1);
+                        const int prow = MODE == 0 ? row & 63 : row;
+                        if (off < kd16 && row0 + prow < plane_rows) {
+                            const uint8_t *src = MODE == 0 ? (row < 64 ? sc0 + (size_t)row * kd16
+                                                                       : sc1 + (size_t)(row - 64) * kd16)
+                                                           : sc0 + (size_t)row * kd16;
+                            cp_async8(raw + kRawCodeBytes + row * 16 + 8 * (ci & 1), src + off);
+                        }
                     }
+                    cp_async_arrive_noinc(&bars->raw_full[rr.stage]);
+                } else {
+                    // 128 rows x eight 2-byte pieces, zeros where there is no scale
+#pragma unroll 8
+                    for (int k = 0; k < (8 * kBM) / 32; k++) {
+                        const int ci = lane + 32 * k, row = ci >> 3, off = 16 * R + 2 * (ci & 7);
+                        const int prow = MODE == 0 ? row & 63 : row;   // row within its plane's box
+                        unsigned short v = 0;
+                        if (off < kd16 && row0 + prow < plane_rows) {
+                            const uint8_t *src = MODE == 0 ? (row < 64 ? sc0 : sc1) : sc0;
+                            v = *reinterpret_cast<const unsigned short *>(src + (size_t)prow * kd16 + off);
+                        }
+                        *reinterpret_cast<unsigned short *>(raw + kRawCodeBytes + row * 16 + 2 * (ci & 7)) = v;
+                    }
+                    mbar_arrive(&bars->raw_full[rr.stage]);
                 }
-                cp_async_arrive_noinc(&bars->raw_full[rr.stage]);
                 rr.next();
             }
         }
@@ -455,20 +487,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Tile t = tiles[cid + tl * ncl];
             const int buf = tl & 1;
             const int e = t.expert;
+            // gate/up: x's staging factor for g, and for u that factor times 2^hexp
+            // of the pair's token (h is stored relative to it; the combine undoes
+            // it); down: routing weight x s_d
             const float *colf = MODE == 0 ? p.ps : p.pw;
             const float cscale = MODE == 0 ? 1.0f : p.down_global[e];
-            float cf[kBN / 128];
+            float cf[kBN / 128], cu[kBN / 128];
 #pragma unroll
             for (int c = 0; c < kBN / 128; c++) {
                 const int col = 128 * c + threadIdx.x;
                 cf[c] = col < t.ntok ? colf[t.pos0 + col] * cscale : 0.0f;
+                if (MODE == 0) cu[c] = col < t.ntok ? cf[c] * p.ph[t.pos0 + col] : 0.0f;
             }
             const bool got = mbar_wait(&bars->acc_full[buf], (acc_phase >> buf) & 1, abort, p.status, 8);
             // The AND-barrier also orders every read of colf_s for the previous
             // tile before the writes below.
             if (!epi_all(got)) break;
 #pragma unroll
-            for (int c = 0; c < kBN / 128; c++) colf_s[128 * c + threadIdx.x] = cf[c];
+            for (int c = 0; c < kBN / 128; c++) {
+                colf_s[128 * c + threadIdx.x] = cf[c];
+                if (MODE == 0) colu_s[128 * c + threadIdx.x] = cu[c];
+            }
             epi_sync();
             acc_phase ^= 1u << buf;
             tc_fence_after();
@@ -480,6 +519,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int il = 16 * warp + (lane & 15);
                 const bool is_gate = lane < 16;
                 const int i0 = t.m0 + kGuCta * rank;
+                // intermediates of this half inside I (a partial last tile when I is
+                // not a multiple of 128 reads the next expert's rows; dropped)
+                const int ni = max(0, min(kGuCta, p.I - i0));
+                const bool row_ok = il < ni;
                 bool fin = true;
 #pragma unroll 1
                 for (int c = 0; c < kChunks; c++) {
@@ -488,11 +531,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // This lane's 16 column factors, in registers before the first
                     // staging store (shared loads after it would wait for it).
                     const int cj0 = is_gate ? 0 : 16;
-                    float xs[16];
+                    float xs[16], xu[16];
 #pragma unroll
                     for (int k = 0; k < 4; k++) {
                         const float4 f = reinterpret_cast<const float4 *>(colf_s + 32 * c + cj0)[k];
                         xs[4 * k] = f.x; xs[4 * k + 1] = f.y; xs[4 * k + 2] = f.z; xs[4 * k + 3] = f.w;
+                        const float4 g = reinterpret_cast<const float4 *>(colu_s + 32 * c + cj0)[k];
+                        xu[4 * k] = g.x; xu[4 * k + 1] = g.y; xu[4 * k + 2] = g.z; xu[4 * k + 3] = g.w;
                     }
                     uint32_t v[32];
                     tmem_ld32(tbase + 32 * c, v);
@@ -506,14 +551,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
                         const float gacc = is_gate ? mine_lo : recv;
                         const float uacc = is_gate ? recv : mine_hi;
-                        const float gv = gacc * sg * xs[j], uv = uacc * su * xs[j];
+                        const float gv = gacc * sg * xs[j], uv = uacc * su * xu[j];
                         const float hf = silu(gv) * uv;
-                        fin &= fits_f16(hf);
+                        fin &= fits_f16(hf) || !row_ok;
                         hs[(cj0 + j) * kGuCta + il] = __float2half_rn(hf);
                     }
                     epi_sync();
-                    store_chunk<kGuCta>(hs, p.h + (size_t)(t.pos0 + 32 * c) * p.I + i0, p.I,
-                                        min(32, t.ntok - 32 * c));
+                    if (ni > 0)
+                        store_chunk<kGuCta>(hs, p.h + (size_t)(t.pos0 + 32 * c) * p.I + i0, p.I,
+                                            min(32, t.ntok - 32 * c), ni);
                 }
                 // h is stored in F16: a value past its range is reported, not hidden
                 if (!fin) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, kNfH | e);
@@ -523,6 +569,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // a fixed order.
                 const int r = 32 * warp + lane;
                 const int m = t.m0 + kBM * rank;
+                const int nr = min(kBM, p.H - m);   // rows of this half inside H
+                const bool row_ok = r < nr;
                 bool fin = true;
                 if (m < p.H) {
 #pragma unroll 1
@@ -544,12 +592,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int j = 0; j < 32; j++) {
                             const float yf = __uint_as_float(v[j]) * cf[j];
-                            fin &= fits_f16(yf);
+                            fin &= fits_f16(yf) || !row_ok;
                             ys[j * kBM + r] = __float2half_rn(yf);
                         }
                         epi_sync();
                         store_chunk<kBM>(ys, p.xh + (size_t)(t.pos0 + 32 * c) * p.H + m, p.H,
-                                         min(32, t.ntok - 32 * c));
+                                         min(32, t.ntok - 32 * c), nr);
                     }
                 }
                 // the per-pair rows w * s_d * y are stored in F16 (see above)

@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(Params p) {
     int *wt = dnb + p.E;                  // [33]
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) cnt_s[e] = p.counts[e];
     __syncthreads();
-    const int mgu = p.I / kGuRows, mdn = cdiv(p.H, kDnRows);
+    const int mgu = cdiv(p.I, kGuRows), mdn = cdiv(p.H, kDnRows);
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
         off_s[e] = cnt_s[e];
         gub[e] = cdiv(cnt_s[e], kBN) * mgu;
@@ -197,10 +197,19 @@ __global__ void __launch_bounds__(256) prep_prefill_kernel(Params p) {
     __syncthreads();
     amax = 0.0f;
     for (int w = 0; w < (int)(blockDim.x >> 5); w++) amax = fmaxf(amax, red[w]);
-    const int sh = (p.act_type == NVFP4_MOE_ACT_INT8) ? 0 : pow2_shift_for(amax);
-    const float xs = (p.act_type == NVFP4_MOE_ACT_INT8) ? p.act_scale[t] : exp2i(-sh);
-    if (threadIdx.x == 0) p.xscale[t] = xs;
-    if (threadIdx.x < p.K) p.ps[spos[threadIdx.x]] = xs;
+    const bool int8 = p.act_type == NVFP4_MOE_ACT_INT8;
+    const int sh = int8 ? 0 : pow2_shift_for(amax);
+    const float xs = int8 ? p.act_scale[t] : exp2i(-sh);
+    // h of this token's pairs is stored times 2^he (the combine divides it out)
+    const int he = h_exp_for(int8 ? 127.0f * xs : amax);
+    if (threadIdx.x == 0) {
+        p.xscale[t] = xs;
+        p.phinv[t] = exp2i(-he);
+    }
+    if (threadIdx.x < p.K) {
+        p.ps[spos[threadIdx.x]] = xs;
+        p.ph[spos[threadIdx.x]] = exp2i(he);
+    }
 #pragma unroll
     for (int i = 0; i < kMaxPer; i++) {
         const int k8 = threadIdx.x + i * blockDim.x;
@@ -258,10 +267,12 @@ __global__ void __launch_bounds__(256) combine_kernel(Params p) {
                 }
             }
         }
+        // the rows were built from h stored times 2^he of this token
+        const float hinv = p.phinv[t];
         bool fin = true;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            acc[i] += sum[i];
+            acc[i] += sum[i] * hinv;
             fin &= isfinite(acc[i]);
         }
         if (!fin) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, kNfOut | t);

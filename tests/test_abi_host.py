@@ -53,8 +53,9 @@ def _weights(align=256):
 
 @pytest.mark.parametrize("dims,code", [
     ((2048, 768, 512, 10, 64), None),            # valid dims: fails later (no device / fake ptrs)
-    ((2048, 700, 512, 10, 64), -2),              # I not a multiple of 128
-    ((2000, 768, 512, 10, 64), -2),              # H not a multiple of 128
+    ((2080, 800, 512, 10, 64), None),            # H, I multiples of 32 (not of 128): valid
+    ((2048, 700, 512, 10, 64), -2),              # I not a multiple of 32
+    ((2000, 768, 512, 10, 64), -2),              # H not a multiple of 32
     ((2048, 768, 8, 10, 64), -2),                # K > E
     ((2048, 768, 512, 17, 64), -2),              # K > 16
     ((2048, 768, 2048, 10, 64), -2),             # E > 1024

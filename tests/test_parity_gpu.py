@@ -216,3 +216,36 @@ def test_f16_range_overflow_is_reported_never_silent(T, which):
         assert st == -7                 # h itself overflows F16 on both paths
     elif T > 8:
         assert st == -7                 # the per-pair F16 rows overflow
+
+
+@pytest.mark.parametrize("T", [3, 8, 300])
+def test_outputs_are_bitwise_reproducible(T):
+    """Both paths add each token's expert rows in a fixed order with no
+    floating-point atomics: the same call twice gives the same bits."""
+    import nvfp4_mixture_experts_03_b200 as nv
+    dims = synth.LayerDims(E=64, H=512, I=384, K=6)
+    layer, logits, x, _ = _case(dims, T, seed=71, zipf=1.1, outliers=True)
+    m = nv.MoELayer.from_layer(layer.to(DEV), top_k=dims.K, max_tokens=max(T, 8))
+    xd, ld = x.to(DEV), logits.to(DEV)
+    a = m.forward(xd, logits=ld).clone()
+    b = m.forward(xd, logits=ld).clone()
+    assert m.status() == 0
+    m.close()
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
+@pytest.mark.parametrize("T", [5, 70])
+@pytest.mark.parametrize("H,I", [(160, 96), (224, 160), (256, 96), (160, 256), (96, 288)])
+def test_hidden_and_inter_multiples_of_32(H, I, T):
+    """H and I that are multiples of 32 but not of 128: K rounds and K steps with a
+    zero-padded tail, partial gate/up and down row tiles, and scale rows that are
+    not 8-byte aligned. The last expert is made popular so the partial tiles at
+    the very end of each plane are reached."""
+    dims = synth.LayerDims(E=6, H=H, I=I, K=2)
+    layer, logits, x, xs = _case(dims, T, seed=81 + H + I)
+    logits[:, dims.E - 1] += 1.5
+    ref, out, dbg, st = _run_both(layer, logits, x, xs, dims.K)
+    assert st == 0
+    assert ref["counts"][dims.E - 1] > 0
+    check_routing(dbg, ref, T, dims.K)
+    assert_close(out, ref["out"], f"H={H} I={I} T={T}")
