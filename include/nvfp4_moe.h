@@ -44,8 +44,9 @@
  *     owned by the caller. The handle BORROWS the weight pointers: they must stay
  *     valid until nvfp4_moe_destroy. The library allocates no device memory
  *     except what nvfp4_moe_create makes: a 256-byte status block and, when
- *     the layer can take the decode kernel, its state (2304 bytes of counters),
- *     kept zero between calls.
+ *     the layer can take the decode kernel, its state, kept zero between calls:
+ *     a counter and a 64-bit copy of the output, 256 + 64 * H bytes (128 KB for
+ *     H = 2048).
  *   - All other scratch lives in the caller's workspace (nvfp4_moe_workspace_bytes).
  *
  * Errors: every call returns 0 (NVFP4_MOE_OK) or a negative nvfp4_moe_status.
@@ -67,15 +68,17 @@
  *   upstream Strata": folding a tiny scale into FP16 activations pushed them
  *   into FP16 subnormals).
  *
- * Decode: calls with T <= 8 run one decode kernel (one CTA per SM) when
- *   H <= 6144 and I <= 6144 (its shared-memory rings must hold at least two items
- *   of each projection: 9 * H and 9 * I bytes each); other layers run small
- *   batches through the grouped-GEMM path. The decode kernel adds each token's
- *   K expert rows in the fixed order j = 0..K-1 and uses no floating-point
- *   atomics, so, like the grouped-GEMM path, it returns the same bits on every
- *   run. Its CTAs wait on one another through counters (bounded). It assumes the
- *   GPU is not shared with other work that keeps SMs busy for long; otherwise
- *   such waits can run out and the call reports NVFP4_MOE_ERR_TIMEOUT.
+ * Decode: calls with T <= 8 run one decode kernel (one CTA per SM) when its
+ *   shared memory (the 8 activation rows at H, plus one CTA's slice of h) fits
+ *   150 KB -- e.g. every layer with H <= 4096 and I <= 2048 at top-k <= 16 and
+ *   <= 512 experts; other layers run small batches through the grouped-GEMM
+ *   path. Each CTA computes gate/up, SwiGLU and the down projection for its own
+ *   slice of the selected experts' intermediates; the slices' partial outputs are
+ *   added as 64-bit integers (value x 2^32, rounded to nearest, so a partial sum
+ *   must stay below 2^31 in magnitude, else the call reports
+ *   NVFP4_MOE_ERR_NONFINITE): integer addition does not depend on the order of the
+ *   adds, so, like the grouped-GEMM path, the decode kernel returns the same bits
+ *   on every run. No CTA waits on another.
  *
  * Threading: a handle may be used from one host thread at a time. Two forward
  *   calls that run concurrently on the GPU must not share a workspace.
@@ -253,16 +256,17 @@ NVFP4_MOE_API int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events
  * for callers that cannot allocate device memory at all, and so cannot create a
  * handle -- nvfp4_moe_create allocates a status block -- or pass a workspace).
  * It runs the same decode path as nvfp4_moe_forward for 1 <= T <= 8 tokens, with
- * its scratch in a 2 MiB array compiled into the library (a file-scope
+ * its scratch in a 1 MiB array compiled into the library (a file-scope
  * __device__ array: every GPU that loads the library holds it until the process
  * exits). dims and weights are checked exactly as by nvfp4_moe_create; io and
  * stream are as for nvfp4_moe_forward. Calls no cudaMalloc/cudaFree.
  *   - T > 8, or a layer outside the decode kernel (see "Decode" above),
  *     returns NVFP4_MOE_ERR_UNSUPPORTED_DIMS; a layer whose decode scratch and
- *     state for this T exceed 2 MiB - 256 bytes returns
- *     NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL (e.g. H = I = 4096 with K = 16 at
- *     T = 8: the FP32 per-pair down rows alone take 2 MiB). Both are checked
- *     before anything is enqueued. T = 0 is a no-op.
+ *     state for this T exceed 1 MiB - 256 bytes would return
+ *     NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL (no layer the decode kernel takes needs
+ *     that much: its state is 64 * H bytes and its shared memory bounds H and
+ *     the expert count). Both are checked before anything is enqueued. T = 0
+ *     is a no-op.
  *   - The first call on a device does a one-time set-up there: it looks up the
  *     array's device address (cudaGetSymbolAddress) and opts the decode kernels
  *     into the shared memory they need (cudaFuncSetAttribute). Make that first

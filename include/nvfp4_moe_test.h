@@ -15,9 +15,9 @@
 extern "C" {
 #endif
 
-/* Decode (T <= 8): CTA 0 never reports that it has read the activations, so
- * every CTA's bounded wait before the down phase runs out (after about 200 ms),
- * the call latches NVFP4_MOE_ERR_TIMEOUT, and the layer's output is not valid.
+/* Decode (T <= 8): CTA 0 never arrives at the grid barrier between the gate/up
+ * and down phases, so every CTA's bounded wait there runs out (after about
+ * 200 ms), the call latches NVFP4_MOE_ERR_TIMEOUT and leaves out unwritten.
  * nvfp4_moe_get_status then returns TIMEOUT and clears the decode state, after
  * which calls with the flag off are correct again. */
 #define NVFP4_MOE_TEST_DECODE_STALL 1
@@ -29,7 +29,7 @@ NVFP4_MOE_API int nvfp4_moe_test_set_flags(nvfp4_moe_t *h, int32_t flags);
 /* The detail word that came with the status the last nvfp4_moe_get_status on h
  * returned (0 when it returned 0). For NVFP4_MOE_ERR_NONFINITE raised by a
  * computed value: (1 << 20) | expert for h, (2 << 20) | expert for a per-pair
- * down row, (3 << 20) | (token or first row) for the output; a token index for a
+ * down row, (3 << 20) | (token or row) for the output; a token index for a
  * routing logit. For NVFP4_MOE_ERR_TIMEOUT: where the wait gave up. Returns 0 for
  * a NULL handle. */
 NVFP4_MOE_API int nvfp4_moe_test_last_detail(const nvfp4_moe_t *h);

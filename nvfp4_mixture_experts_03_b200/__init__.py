@@ -144,8 +144,8 @@ def nvfp4_moe_set_phase_events(handle: int, events) -> int:
 
 
 def nvfp4_moe_test_set_flags(handle: int, flags: int) -> int:
-    """Test hook (include/nvfp4_moe_test.h): TEST_DECODE_STALL makes decode's bounded
-    waits run out, so the call latches TIMEOUT."""
+    """Test hook (include/nvfp4_moe_test.h): TEST_DECODE_STALL makes decode's grid
+    barrier wait run out, so the call latches TIMEOUT."""
     return lib().nvfp4_moe_test_set_flags(C.c_void_p(handle), C.c_int32(flags))
 
 
@@ -160,7 +160,7 @@ def nvfp4_moe_test_fail_alloc(n: int) -> None:
 
 
 def nvfp4_moe_forward_decode_static(dims: Dims, weights: Weights, io: IO, stream: int) -> int:
-    """Allocation-free decode (T <= 8): scratch is a 2 MiB array inside the library,
+    """Allocation-free decode (T <= 8): scratch is a 1 MiB array inside the library,
     shared by every call on the device -- serialise calls. No handle, no workspace."""
     return lib().nvfp4_moe_forward_decode_static(C.byref(dims), C.byref(weights), C.byref(io),
                                                  C.c_void_p(stream))

@@ -30,10 +30,10 @@ enum : int { kStatusCode = 0, kStatusDetail = 1, kStatusWords = 64 };
 
 // Per-call routing/tile counters kept in the workspace (int32 words).
 enum : int { kCntTilesGu = 0, kCntTilesDn = 1, kCntUniq = 2, kCntWords = 64 };
-// Decode state (per handle, int32 words, zero between launches). kDsDone: CTAs
-// whose down rows are written; kDsExit: CTAs done; kDsReady + u: finished gate/up
-// items of used expert u (u < 128).
-enum : int { kDsDone = 0, kDsExit = 1, kDsReady = 2, kDsWords = 2 + 128 };
+// Decode state (per handle, int32 counters, zero between launches): kDsArrive:
+// CTAs past the gate/up phase (the grid barrier); kDsExit: CTAs done.
+enum : int { kDsArrive = 0, kDsExit = 1, kDsInts = 64 };
+inline size_t decode_state_bytes() { return (size_t)kDsInts * 4; }
 
 struct Tile {  // one grouped-GEMM tile
     int32_t expert;   // expert id
@@ -75,7 +75,6 @@ struct Params {
     float *ph;                 // [P] prefill: 2^hexp of the pair's token at each position
     float *phinv;              // [T] prefill: 2^-hexp per token
     Tile *tiles_gu, *tiles_dn;
-    float *ybuf;               // decode: [P][H] FP32 w * s_d * y per pair position
     __half *xh;                // prefill: [P][H] F16 activations per pair position, then the
                                // down projection's w * s_d * y per pair (F16)
     __half *h;                 // [P][I]
@@ -87,7 +86,8 @@ struct Params {
     int32_t nch;               // routing chunks
     int32_t max_tiles_gu, max_tiles_dn;
     int32_t *dstate;           // decode: counters (kDs*), zero between launches
-    int32_t dec_n1, dec_n2;    // decode: ring slots for gate/up and for down items
+    int32_t dec_union;         // decode: bytes of the phase-shared dynamic shared memory
+    int32_t dec_raw;           // decode: raw activations copied to shared memory first
     int32_t test_flags;        // NVFP4_MOE_TEST_* (test hooks; 0 in production)
 };
 
@@ -395,11 +395,12 @@ void launch_prep_prefill(const Params &p, cudaStream_t s);
 void launch_combine(const Params &p, cudaStream_t s);   // prefill: per-token sum of the K pair rows
 cudaError_t launch_decode(const Params &p, cudaStream_t s);   // the whole T <= 8 layer
 int decode_grid();                                 // CTAs of the decode kernel (one per SM)
+constexpr int kDecWarpsPerCta = 16;                // warps of a decode CTA
 // Whether the decode kernel's shared-memory plan holds layers of these dims (else
 // small batches take the grouped-GEMM path).
-bool decode_fits(int H, int I);
-// Bytes of the decode state (kDsWords counters).
-inline size_t decode_state_bytes() { return ((size_t)kDsWords * 4 + 255) & ~size_t(255); }
+bool decode_fits(int H, int I, int K, int E);
+size_t decode_union_bytes(int T, int K, int H, int I, int act_type, bool raw);
+bool decode_raw_staged(int T, int K, int E, int H, int I, int act_type);
 // mode 0: gate/up + SwiGLU, map_b = F16 activations [P][H]; mode 1: down, map_b =
 // h [P][I]; both 64 x 64 boxes
 // Tensor maps of the packed E2M1 code planes (bytes; 128-byte x 64-row boxes for

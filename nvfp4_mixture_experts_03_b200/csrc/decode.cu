@@ -5,80 +5,87 @@
 // the measurements) and note that a decode round is bound by moving expert
 // bytes ("Strata NVFP4" README, "Limits"). On B200 every expert is resident in
 // HBM, so decode is a pure HBM stream whose time is set by how early the weight
-// copies start, how many bytes are in flight and how evenly they are spread.
+// loads start, how many are in flight, and how few round trips lie between them.
 //
-// One kernel per layer, one CTA per SM (16 consumer warps + 2 producer warps),
-// launched with programmatic dependent launch:
+// One kernel per layer, one 16-warp CTA per SM, launched with programmatic
+// dependent launch:
 //   routing: every CTA routes the <= 8 tokens itself (warp top-k per token, then
-//     the <= 128 (token, slot) pairs ranked by (expert, token)), so no CTA waits
-//     for another before its weight stream starts;
-//   work: phase-1 items (used expert u, 8 intermediates: 8 gate + 8 up rows, all
-//     of K = H) and phase-2 items (u, 16 hidden rows, all of K = I) are cut into
-//     equal contiguous ranges, one range of each per CTA;
-//   producer warps: as soon as routing is done, one copies the CTA's phase-1
-//     items and the other its phase-2 items into two shared-memory rings with 1-D
-//     bulk copies (each item's code rows and scale rows are contiguous blocks
-//     of each projection), so the down weights stream in while gate/up computes;
-//   consumer warps: each warp owns fixed 128-wide K rounds of an item, and holds
-//     the activations (phase 1) or the expert's h rows (phase 2) of those rounds
-//     in registers as mma.sync B fragments. A group of warps covers one item's K;
-//     their FP32 partial sums meet in shared memory and are added in a fixed warp
-//     order. Phase 1 ends in SwiGLU and the F16 h row; each finished item counts
-//     towards its expert's ready count. Phase 2 waits for its expert's count,
-//     writes w * s_d * y per pair as FP32 rows, and the CTA that completes a block
-//     of 16 hidden rows (one item per used expert) adds each token's K rows in the
-//     fixed order j = 0..K-1 into out. No floating-point atomics: the output is
-//     the same bits on every run.
-// Cross-CTA waits (expert ready counts, the count of CTAs that have read the
-// activations, which out may alias) are bounded; the last CTA to finish resets
-// the counters for the next launch.
+//     positions by counting), and stages the activations as F16 in shared
+//     memory (its first weight loads are already in flight by then);
+//   gate/up + SwiGLU: the flattened space of (used expert, 8 intermediates)
+//     granules is cut into equal contiguous ranges, one per CTA; a CTA splits
+//     its (granule, 128-wide K round) units evenly over its warps, sums a granule
+//     split between warps in shared memory in warp order, and stores h (F16 with
+//     a per-token power-of-two range exponent) at each pair's position;
+//   one grid barrier (bounded wait): every h is stored, every CTA has read the
+//     activations (out may alias them);
+//   down + weighted combine: each CTA owns whole 16-row blocks of out and, for
+//     every used expert, streams those rows of the expert's down matrix (whole
+//     rows: contiguous bytes, which DRAM serves about twice as fast as a column
+//     slice of the same size), with every pair's h row staged in shared memory.
+//     Per row block the experts are summed in registers in ascending order
+//     (scaled by w * s_d), a block split between warps in warp order, and the
+//     rows of out are stored once, in FP32.
+// Determinism: every sum runs in a fixed order and no value is added by an
+// atomic, so the result is the same bits on every run.
 // Arithmetic: each weight is decoded exactly to F16 (E2M1 -> F16 conversion
-// times its E4M3 group scale: at most 6 significant bits) and fed to mma.sync
-// m16n8k16 with the token slots as N, FP32 accumulation; the tensor scale and
-// the per-token activation scale are applied to the FP32 result.
+// times its E4M3 group scale: at most 6 significant bits, exact in F16) and fed
+// to mma.sync m16n8k16 with the token slots as N, FP32 accumulation; the tensor
+// scale and the per-token activation scale are applied to the FP32 result.
 //
 // Fragment mapping (m16n8k16, A row-major, B col-major): thread (g = lane/4,
-// q = lane%4) holds A rows g and g+8; per 128-wide K round it reads 16
-// contiguous code bytes of each row (byte offset 64*r + 16*q). Mma step s of
-// round r uses physical K 128r + 32q + 4s + {0,1,2,3} for logical K {2q, 2q+1,
-// 2q+8, 2q+9}; the B fragments use the same permutation, so every dot product
-// is the plain one. H and I need only be multiples of 32: a 32-wide piece of a
-// round past the end is zero on both sides.
+// q = lane%4) holds rows g and g+8. It loads 16 contiguous code bytes of each
+// row per 128-wide K round (byte offset 64*r + 16*q), so a warp reads whole
+// 32-byte sectors. Mma step s of round r uses physical K 128r + 32q + 4s +
+// {0,1,2,3} for logical K {2q, 2q+1, 2q+8, 2q+9}; the activations and h use the
+// same permutation, so every dot product is the plain one. H and I need only be
+// multiples of 32: a 32-wide piece of a round past the end is zero on both sides.
 #include "common.cuh"
 #include "route_common.cuh"
 
 namespace nvmoe {
 
-// Timeline marks for profiling builds (compiled with NVMOE_DEC_TRACE): the
-// global timer per CTA at a few points of the layer; nothing otherwise.
-#ifdef NVMOE_DEC_TRACE
-__device__ unsigned long long g_dec_trace[1024][8];
-#define DEC_MARK(i) (g_dec_trace[blockIdx.x][(i)] = globaltimer())
-#else
-#define DEC_MARK(i) ((void)0)
-#endif
+__device__ inline uint4 ldg_stream(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
 
 __device__ inline void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ inline void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
-constexpr int kDecCW = 16;                          // consumer warps
-constexpr int kDecThreads = (kDecCW + 2) * 32;      // + two producer warps (one per ring)
-constexpr int kMaxRW = 3;                           // K rounds of B fragments a warp holds
+// Eight mma steps of one 128-wide K round: A rows (g: ca, g+8: cb) as 16 code
+// bytes each with their two group scales; B from `bfrag(s)`.
+template <class BF>
+__device__ inline void round_mma(float (&acc)[4], const uint4 &ca, const uint4 &cb, uint32_t sa,
+                                 uint32_t sb, BF bfrag) {
+    const uint32_t sa0 = e4m3_to_f16x2_bcast(sa & 0xFF), sa1 = e4m3_to_f16x2_bcast(sa >> 8);
+    const uint32_t sb0 = e4m3_to_f16x2_bcast(sb & 0xFF), sb1 = e4m3_to_f16x2_bcast(sb >> 8);
+    const uint32_t wa[4] = {ca.x, ca.y, ca.z, ca.w}, wb[4] = {cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+    for (int w = 0; w < 4; w++) {
+        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+        e2m1x8_to_f16(wa[w], a0, a1, a2, a3);   // bytes 4w..4w+3 of row g
+        e2m1x8_to_f16(wb[w], b0, b1, b2, b3);   // same bytes of row g+8
+        const uint32_t s_a = w < 2 ? sa0 : sa1, s_b = w < 2 ? sb0 : sb1;
+        uint32_t x0, x1;
+        bfrag(2 * w, x0, x1);
+        mma_16816(acc, hmul2(a0, s_a), hmul2(b0, s_b), hmul2(a1, s_a), hmul2(b1, s_b), x0, x1);
+        bfrag(2 * w + 1, x0, x1);
+        mma_16816(acc, hmul2(a2, s_a), hmul2(b2, s_b), hmul2(a3, s_a), hmul2(b3, s_b), x0, x1);
+    }
+}
+
+constexpr int kDecWarps = kDecWarpsPerCta;
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kGuRounds = 4;   // gate/up: 128-wide K rounds of loads one warp holds per chunk
+constexpr int kDnUnits = 3;    // down: (16 rows, expert, 128-wide K round) units one warp holds per chunk
 constexpr int kMaxPairs = NVFP4_MOE_DECODE_MAX_T * NVFP4_MOE_MAX_TOPK;  // 128
 constexpr int kSlots = NVFP4_MOE_DECODE_MAX_T;
-constexpr int kPartBytes = kDecCW * 2 * 32 * 16;    // partial sums: [warp][2 buffers][lane] float4
-constexpr int kBarConsumers = 15;                   // named barrier over the 16 consumer warps
-constexpr uint64_t kDecWaitNs = 200000000ull;
-constexpr uint64_t kDecDrainNs = 200000000ull;
-constexpr int kDecSmemBudget = 208 * 1024;          // dynamic shared memory the plan may use (+ about 12 KB static)
 
-// Warps per item for a projection of NR K rounds: the fewest (2, 4, 8 or 16)
-// that leave each warp at most kMaxRW rounds; 0 when NR is too large.
-__host__ __device__ inline int dec_group_warps(int nr) {
-    for (int wg = 2; wg <= kDecCW; wg *= 2)
-        if (cdiv(nr, wg) <= kMaxRW) return wg;
-    return 0;
-}
+constexpr uint64_t kDecWaitNs = 200000000ull;   // grid barrier wait limit (200 ms)
 
 // Per-CTA routing state of the decode kernel.
 struct DecRoute {
@@ -87,9 +94,13 @@ struct DecRoute {
     int pos[kMaxPairs];             // position of pair q (grouped by expert, then token)
     int sorted_e[kMaxPairs];        // expert at each position
     int uniq[kMaxPairs];            // used experts, ascending
+    int uoff[kMaxPairs + 1];        // first position of each used expert; uoff[U] = P
     int upos[kMaxPairs * kSlots];   // pair position of (used expert, token), -1 if absent
     float uw[kMaxPairs * kSlots];   // routing weight of (used expert, token)
+    float dw[kMaxPairs * kSlots];   // w * s_d * 2^-hexp of (used expert, token), 0 if absent
     unsigned amax[kSlots];          // per-token activation amax (FP32 bits)
+    float xsc[kSlots];              // per-token factor that undoes the F16 staging scale
+    int hexp[kSlots];               // per-token exponent h is stored with (h_exp_for)
     int wtot[33];                   // block scan scratch
     int U;
 };
@@ -101,9 +112,9 @@ struct DecRoute {
 // exclusive scan over the experts gives each expert's first position and its
 // index among the used experts; a pair's position is its expert's first position
 // plus the number of earlier tokens in the mask. `ex` and `sc` are E ints of
-// shared scratch each.
-template <int NPER>
-__device__ void cta_route(const Params &p, DecRoute &R, bool report, int *ex, int *sc) {
+// shared scratch each. Warps kSlots.. (which route no token) run `side` meanwhile.
+template <int NPER, class Side>
+__device__ void cta_route(const Params &p, DecRoute &R, bool report, int *ex, int *sc, Side side) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = p.T * p.K, E = p.E;
     for (int i = threadIdx.x; i < kMaxPairs * kSlots; i += blockDim.x) R.upos[i] = -1;
@@ -127,6 +138,8 @@ __device__ void cta_route(const Params &p, DecRoute &R, bool report, int *ex, in
             R.w[warp * p.K + lane] = w;
             atomicAdd(&ex[id], 1 + (1 << (16 + warp)));
         }
+    } else if (warp >= kSlots) {
+        side();
     }
     __syncthreads();
     // pairs before each expert (bits 0..15) and used experts before it (16..)
@@ -145,9 +158,15 @@ __device__ void cta_route(const Params &p, DecRoute &R, bool report, int *ex, in
         R.sorted_e[rank] = e;
         R.upos[u * kSlots + t] = rank;
         R.uw[u * kSlots + t] = R.w[q];
-        if (within == 0) R.uniq[u] = e;
+        if (within == 0) {
+            R.uniq[u] = e;
+            R.uoff[u] = rank;
+        }
     }
-    if (threadIdx.x == 0) R.U = total >> 16;
+    if (threadIdx.x == 0) {
+        R.U = total >> 16;
+        R.uoff[total >> 16] = P;
+    }
     __syncthreads();
 }
 
@@ -189,167 +208,206 @@ __device__ void publish_route(const Params &p, const DecRoute &R) {
     if (threadIdx.x == 0) p.cnt[kCntUniq] = R.U;
 }
 
-// Eight mma steps of one 128-wide K round: A rows (g: ca, g+8: cb) as 16 code
-// bytes each with their two group scales; B fragments of the round in bx.
-__device__ inline void round_mma(float (&acc)[4], const uint4 &ca, const uint4 &cb, uint32_t sa,
-                                 uint32_t sb, const uint4 (&bx)[4]) {
-    const uint32_t sa0 = e4m3_to_f16x2_bcast(sa & 0xFF), sa1 = e4m3_to_f16x2_bcast(sa >> 8);
-    const uint32_t sb0 = e4m3_to_f16x2_bcast(sb & 0xFF), sb1 = e4m3_to_f16x2_bcast(sb >> 8);
-    const uint32_t wa[4] = {ca.x, ca.y, ca.z, ca.w}, wb[4] = {cb.x, cb.y, cb.z, cb.w};
-#pragma unroll
-    for (int w = 0; w < 4; w++) {
-        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-        e2m1x8_to_f16(wa[w], a0, a1, a2, a3);   // bytes 4w..4w+3 of row g
-        e2m1x8_to_f16(wb[w], b0, b1, b2, b3);   // same bytes of row g+8
-        const uint32_t s_a = w < 2 ? sa0 : sa1, s_b = w < 2 ? sb0 : sb1;
-        const uint4 &x = bx[w];                 // steps 2w and 2w+1
-        mma_16816(acc, hmul2(a0, s_a), hmul2(b0, s_b), hmul2(a1, s_a), hmul2(b1, s_b), x.x, x.y);
-        mma_16816(acc, hmul2(a2, s_a), hmul2(b2, s_b), hmul2(a3, s_a), hmul2(b3, s_b), x.z, x.w);
+// A CTA's share of the gate/up phase: granules [gb, ge) of the flattened (used
+// expert, 8 intermediates) space.
+struct DecPlan {
+    int gb, ge;
+    int ok;     // the grid barrier completed
+    int last;   // this CTA finished last (resets the counters)
+};
+
+// Gate/up weights of one warp's chunk: rows g (gate) and g+8 (up), up to
+// kGuRounds rounds.
+struct GuBuf {
+    uint4 ca[kGuRounds], cb[kGuRounds];
+    uint32_t s[kGuRounds];   // row g's two scale bytes in bits 0..15, row g+8's in 16..31
+};
+
+// A run of at most kGuRounds consecutive K rounds of one granule (CTA-local).
+struct Chunk {
+    int item, r0, r1;   // r1 == 0: none
+};
+
+// Next chunk of the unit range [x, end) (units = item * R + round); advances x.
+__device__ inline Chunk take_chunk(int &x, int end, int R) {
+    Chunk c{0, 0, 0};
+    if (x < end) {
+        c.item = x / R;
+        c.r0 = x - c.item * R;
+        c.r1 = min(min(R, c.r0 + kGuRounds), end - c.item * R);
+        x = c.item * R + c.r1;
     }
+    return c;
 }
 
-// Code bytes and scales of A rows `rowa` and `rowb` for round r of an item held
-// in a ring slot: codes [16 rows][kb] bytes, then scales [16 rows][kb/8]; the
-// 16-byte pieces of the round past a row's end (kb = K/2 bytes) are zero.
-__device__ inline void slot_round(const uint8_t *slot, int kb, int rowa, int rowb, int r, int q,
-                                  uint4 &ca, uint4 &cb, uint32_t &sa, uint32_t &sb) {
-    const int off = 64 * r + 16 * q;
-    if (off < kb) {
-        ca = *reinterpret_cast<const uint4 *>(slot + (size_t)rowa * kb + off);
-        cb = *reinterpret_cast<const uint4 *>(slot + (size_t)rowb * kb + off);
-        const uint8_t *sc = slot + 16 * (size_t)kb;
-        const int soff = 8 * r + 2 * q, sk = kb / 8;
-        sa = *reinterpret_cast<const unsigned short *>(sc + rowa * sk + soff);
-        sb = *reinterpret_cast<const unsigned short *>(sc + rowb * sk + soff);
-    } else {
-        ca = cb = make_uint4(0, 0, 0, 0);
-        sa = sb = 0;
-    }
-}
-
-// 1-D bulk copy global -> this CTA's shared memory, completing on `bar` (bytes
-// counted by the barrier's transaction count). Both addresses 16-byte aligned,
-// size a multiple of 16. No multicast.
-__device__ inline void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ inline void named_bar(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// Warp-uniform bounded mbarrier wait of the consumers.
-__device__ inline bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int32_t *status,
-                                 int where) {
-    const bool ok = mbar_wait(bar, parity, abort, status, where, kDecWaitNs);
-    return __all_sync(0xffffffffu, ok);
-}
-
-// This thread's 32 activations of token t at K offsets k0..k0+31 (k0 < H) as raw
-// bits: BF16 in all four words (FP32 input rounded to BF16 on load), int8 in the
-// first two.
-__device__ inline void load_x32(const Params &p, int t, int k0, uint4 (&v)[4]) {
-    const size_t off = (size_t)t * p.H + k0;
-    if (p.act_type == NVFP4_MOE_ACT_BF16) {
-        const uint4 *s = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.act) + off);
+// Weight loads of rounds [c.r0, c.r1) of granule P.gb + c.item; 16-byte pieces
+// past the row's end (H not a multiple of 128) are zero, with zero scales.
+__device__ inline void gu_issue(const Params &p, const DecRoute &R, const DecPlan &P, const Chunk &c,
+                                int g, int q, GuBuf &b) {
+    if (c.r1 == 0) return;
+    const int per_u = p.I / 8, gi = P.gb + c.item, u = gi / per_u;
+    const size_t ra = (size_t)R.uniq[u] * p.I + (gi - u * per_u) * 8 + g;
+    const int kb = p.H / 2;
+    const uint8_t *ca_p = p.gate_codes + ra * kb, *cb_p = p.up_codes + ra * kb;
+    const uint8_t *sa_p = p.gate_scales + ra * (p.H / 16), *sb_p = p.up_scales + ra * (p.H / 16);
 #pragma unroll
-        for (int i = 0; i < 4; i++) v[i] = __ldg(s + i);
-    } else if (p.act_type == NVFP4_MOE_ACT_INT8) {
-        const uint4 *s = reinterpret_cast<const uint4 *>(static_cast<const int8_t *>(p.act) + off);
-        v[0] = __ldg(s);
-        v[1] = __ldg(s + 1);
-        v[2] = v[3] = make_uint4(0, 0, 0, 0);
-    } else {
-        // out may alias act (residual stream): plain loads, not the read-only path
-        const float4 *s = reinterpret_cast<const float4 *>(static_cast<const float *>(p.act) + off);
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            const float4 a = s[2 * i], b = s[2 * i + 1];
-            const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            uint32_t w[4];
-#pragma unroll
-            for (int j = 0; j < 4; j++)
-                w[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * j])) |
-                       ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * j + 1])) << 16);
-            v[i] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-    }
-}
-
-__device__ inline float raw_amax(const uint4 (&v)[4]) {   // BF16 words
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            m = fmaxf(m, fabsf(__uint_as_float(w[j] << 16)));
-            m = fmaxf(m, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
-        }
-    }
-    return m;
-}
-
-// Raw activations -> F16 B fragments in place: BF16 scaled by 2^sh (exact), or
-// int8 codes (exact in F16).
-__device__ inline void to_f16_frags(bool int8, int sh, uint4 (&v)[4]) {
-    if (int8) {
-        const uint32_t w[8] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w};
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            float f[8];
-#pragma unroll
-            for (int j = 0; j < 8; j++) f[j] = (float)(int8_t)(w[2 * i + (j >> 2)] >> (8 * (j & 3)));
-            v[i] = pack8_f16(f, 0);
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-            float f[8];
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                f[2 * j] = __uint_as_float(w[j] << 16);
-                f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    for (int j = 0; j < kGuRounds; j++) {
+        const int r = c.r0 + j;
+        if (r < c.r1) {
+            if (64 * r + 16 * q < kb) {
+                b.ca[j] = ldg_stream(ca_p + 64 * r + 16 * q);
+                b.cb[j] = ldg_stream(cb_p + 64 * r + 16 * q);
+                b.s[j] = (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sa_p + 8 * r + 2 * q)) |
+                         ((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sb_p + 8 * r + 2 * q)) << 16);
+            } else {
+                b.ca[j] = b.cb[j] = make_uint4(0, 0, 0, 0);
+                b.s[j] = 0;
             }
-            v[i] = pack8_f16(f, sh);
         }
     }
 }
 
-// Per-token factors from the routing state: the one that undoes the F16 staging
-// of token t's activations (2^-shift, or its int8 scale), and the exponent by
-// which its h values are stored (h_exp_for).
-__device__ inline float token_xscale(const Params &p, const DecRoute &R, int t) {
-    return p.act_type == NVFP4_MOE_ACT_INT8 ? __ldg(p.act_scale + t)
-                                            : exp2i(-pow2_shift_for(__uint_as_float(R.amax[t])));
-}
-__device__ inline int token_hexp(const Params &p, const DecRoute &R, int t) {
-    return h_exp_for(p.act_type == NVFP4_MOE_ACT_INT8 ? 127.0f * __ldg(p.act_scale + t)
-                                                      : __uint_as_float(R.amax[t]));
+// h of granule P.gb + j for this thread's intermediate (row g) and token slots
+// 2q, 2q+1 whose token chose the expert, from the granule's full sums (gate: v.x,
+// v.y; up: v.z, v.w), stored F16 at the pair's position.
+__device__ inline void swiglu_store(const Params &p, const DecRoute &R, const DecPlan &P,
+                                    const float *gsc, int j, float4 v, int g, int q, int &bad) {
+    const int per_u = p.I / 8, gi = P.gb + j, u = gi / per_u, e = R.uniq[u];
+    const int i = (gi - u * per_u) * 8 + g;
+    const float sg = gsc[e], su = gsc[p.E + e];
+    const float gs[2] = {v.x, v.y}, us[2] = {v.z, v.w};
+#pragma unroll
+    for (int c = 0; c < 2; c++) {
+        const int slot = 2 * q + c;
+        const int pos = slot < p.T ? R.upos[u * kSlots + slot] : -1;
+        if (pos >= 0) {
+            const float gv = gs[c] * sg * R.xsc[slot], uv = us[c] * su * R.xsc[slot];
+            const float hf = silu(gv) * uv * exp2i(R.hexp[slot]);
+            if (!fits_f16(hf)) bad = e;
+            p.h[(size_t)pos * p.I + i] = __float2half_rn(hf);
+        }
+    }
 }
 
-// Non-blocking release increment: orders this thread's earlier writes (and those
-// it has synchronised with) before the count changes; the thread does not wait.
-__device__ inline void red_release_add(int32_t *p, int v) {
-    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+// Down weights of one warp's chunk: kDnUnits units (16-row block, used expert,
+// 128-wide K round), rows g and g+8, 16 code bytes and two scale bytes each.
+struct DnBuf {
+    uint4 ca[kDnUnits], cb[kDnUnits];
+    uint32_t s[kDnUnits];   // as in GuBuf
+};
+
+// Position of a down unit of the CTA (row blocks rb0.., U experts, R2 rounds
+// each): row block (CTA-local), used expert, round; stepped without division.
+struct DnCur {
+    int rbl, u, r;
+};
+__device__ inline DnCur dn_cur(int x, int U, int R2) {
+    DnCur c;
+    const int per_rb = U * R2;
+    c.rbl = x / per_rb;
+    const int rem = x - c.rbl * per_rb;
+    c.u = rem / R2;
+    c.r = rem - c.u * R2;
+    return c;
 }
-__device__ inline int ld_acquire(const int32_t *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
+__device__ inline void dn_next(DnCur &c, int U, int R2) {
+    if (++c.r == R2) {
+        c.r = 0;
+        if (++c.u == U) {
+            c.u = 0;
+            c.rbl++;
+        }
+    }
 }
 
-// Bounded wait until *word >= target (one thread, acquire); latches TIMEOUT on
-// give-up.
+// Loads of the n <= kDnUnits down units from c on; 16-byte pieces past the row's
+// end (I not a multiple of 128) are zero, with zero scales.
+__device__ inline void dn_issue(const Params &p, const DecRoute &R, int rb0, DnCur c, int n, int g, int q,
+                                DnBuf &b) {
+    const int H = p.H, I = p.I, R2 = cdiv(I, 128), U = R.U;
+#pragma unroll
+    for (int j = 0; j < kDnUnits; j++) {
+        if (j < n) {
+            if (64 * c.r + 16 * q < I / 2) {
+                const size_t ra = (size_t)R.uniq[c.u] * H + 16 * (rb0 + c.rbl) + g;
+                const uint8_t *cp = p.down_codes + ra * (I / 2) + 64 * c.r + 16 * q;
+                const uint8_t *sp = p.down_scales + ra * (I / 16) + 8 * c.r + 2 * q;
+                b.ca[j] = ldg_stream(cp);
+                b.cb[j] = ldg_stream(cp + 8 * (I / 2));
+                b.s[j] = (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sp)) |
+                         ((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sp + 8 * (I / 16))) << 16);
+            } else {
+                b.ca[j] = b.cb[j] = make_uint4(0, 0, 0, 0);
+                b.s[j] = 0;
+            }
+            dn_next(c, U, R2);
+        }
+    }
+}
+
+// out rows 16 rb + g and + 8, token slots 2q, 2q+1 < T, from this thread's sums.
+__device__ inline void store_out(const Params &p, int rb, const float4 &v, int g, int q, int &bad) {
+    const float f[4] = {v.x, v.y, v.z, v.w};   // (row g: slots 2q, 2q+1), (row g+8: same)
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const int slot = 2 * q + (k & 1), row = 16 * rb + g + 8 * (k >> 1);
+        if (slot < p.T) {
+            const size_t o = (size_t)slot * p.H + row;
+            const float r = p.out_add ? p.out[o] + f[k] : f[k];
+            if (!isfinite(r)) bad = row;
+            p.out[o] = r;
+        }
+    }
+}
+
+// Latches NONFINITE (detail: stage | expert or row) if any lane of the warp saw
+// a bad value.
+__device__ inline void warp_report(const Params &p, int bad, int stage) {
+    const unsigned m = __ballot_sync(0xffffffffu, bad >= 0);
+    if (m) {
+        const int v = __shfl_sync(0xffffffffu, bad, __ffs(m) - 1);
+        if ((threadIdx.x & 31) == 0) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, stage | v);
+    }
+}
+
+__device__ inline void cp_async16(void *smem, const void *gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+                 : "memory");
+}
+
+// Raw activation bytes per token held in shared memory (0: FP32 input, which is
+// read from global memory instead).
+__host__ __device__ inline int raw_act_bytes(int act_type, int H) {
+    return act_type == NVFP4_MOE_ACT_BF16 ? 2 * H : (act_type == NVFP4_MOE_ACT_INT8 ? H : 0);
+}
+
+// Eight activations of token t (group k8) as FP32, from the shared raw copy when
+// there is one, else from global memory.
+__device__ inline void act8(const Params &p, const uint8_t *raw, int t, int k8, float (&v)[8]) {
+    if (!raw) {
+        load_act8(p, t, k8, v);
+    } else if (p.act_type == NVFP4_MOE_ACT_BF16) {
+        const uint4 u = reinterpret_cast<const uint4 *>(raw + (size_t)t * 2 * p.H)[k8];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    } else {
+        const uint2 u = reinterpret_cast<const uint2 *>(raw + (size_t)t * p.H)[k8];
+        const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+        for (int i = 0; i < 8; i++) v[i] = (float)(int8_t)(w[i >> 2] >> (8 * (i & 3)));
+    }
+}
+
+// Bounded wait until *word >= target (one thread); latches TIMEOUT on give-up.
 __device__ inline bool wait_geq(const int32_t *word, int target, int32_t *status, int where) {
-    if (ld_acquire(word) >= target) return true;
+    const volatile int32_t *v = word;
+    if (*v >= target) return true;
     const uint64_t t0 = globaltimer();
-    while (ld_acquire(word) < target) {
+    while (*v < target) {
         __nanosleep(32);
         if (globaltimer() - t0 > kDecWaitNs) {
             latch_status(status, NVFP4_MOE_ERR_TIMEOUT, where);
@@ -359,340 +417,337 @@ __device__ inline bool wait_geq(const int32_t *word, int target, int32_t *status
     return true;
 }
 
-// The group's partial sums of an item, added in warp order (deterministic).
-__device__ inline float4 group_sum(const float4 *part, int w0, int wg, int buf, int lane) {
-    float4 s = part[((size_t)w0 * 2 + buf) * 32 + lane];
-    for (int w = 1; w < wg; w++) {
-        const float4 o = part[((size_t)(w0 + w) * 2 + buf) * 32 + lane];
-        s.x += o.x;
-        s.y += o.y;
-        s.z += o.z;
-        s.w += o.w;
-    }
-    return s;
+// Row strides (F16 elements) of the activation tile and of the staged h rows:
+// the K rounds rounded up, plus a few elements so that rows fall in different
+// banks.
+__host__ __device__ inline int dec_ld1(int H) { return cdiv(H, 128) * 128 + 4; }
+__host__ __device__ inline int dec_ld2(int I) { return cdiv(I, 128) * 128 + 8; }
+
+// [a, b) = worker w's share of n units when W workers split them evenly in
+// contiguous ranges.
+__device__ inline void share(int n, int w, int W, int &a, int &b) {
+    a = (int)((long long)n * w / W);
+    b = (int)((long long)n * (w + 1) / W);
+}
+
+// The warp (of W) whose share of n units holds unit x.
+__device__ inline int owner(int n, int W, int x) {
+    int w = (int)(((long long)x * W) / n);   // close; fix up against the exact shares
+    int a, b;
+    share(n, w, W, a, b);
+    while (x < a) share(n, --w, W, a, b);
+    while (x >= b) share(n, ++w, W, a, b);
+    return w;
 }
 
 template <int NPER>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) {
-    extern __shared__ __align__(128) uint8_t dsm[];
+    extern __shared__ __align__(16) uint8_t dsm[];
     __shared__ DecRoute R;
-    __shared__ int s_abort, s_ok;
-    const int H = p.H, I = p.I, T = p.T, K = p.K;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gq = lane >> 2, q = lane & 3;
-    const int N1 = p.dec_n1, N2 = p.dec_n2;
-    const int S1 = 9 * H, S2 = 9 * I;             // bytes of one phase-1 / phase-2 item
-    const int NR1 = cdiv(H, 128), NR2 = cdiv(I, 128);
-    const int WG1 = dec_group_warps(NR1), WG2 = dec_group_warps(NR2);
-    float4 *part = reinterpret_cast<float4 *>(dsm);
-    uint8_t *ringA = dsm + kPartBytes;
-    uint8_t *ringB = ringA + (size_t)N1 * S1;
-    uint64_t *full = reinterpret_cast<uint64_t *>(ringB + (size_t)N2 * S2);
-    uint64_t *empty = full + N1 + N2;
-    volatile int *abort = &s_abort;
+    __shared__ DecPlan P;
+    const int H = p.H, I = p.I, T = p.T;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int ld1 = dec_ld1(H), ld2 = dec_ld2(I);
+    const int raw_bytes = p.dec_raw ? T * raw_act_bytes(p.act_type, H) : 0;
+    // gate/up phase: [8][ld1] F16 activations, raw activations, split-granule parts;
+    // down phase (same storage): [P + 1][ld2] h rows (row P: zeros), split-row-block parts
+    __half *xs = reinterpret_cast<__half *>(dsm);
+    uint8_t *raw = reinterpret_cast<uint8_t *>(xs + kSlots * ld1);
+    float4 *part1 = reinterpret_cast<float4 *>(raw + raw_bytes);
+    __half *hs = reinterpret_cast<__half *>(dsm);
+    float4 *part2 = reinterpret_cast<float4 *>(hs + (size_t)(p.T * p.K + 1) * ld2);
+    int *scratch = reinterpret_cast<int *>(dsm + p.dec_union);   // routing: 2E ints
+    float *gsc = reinterpret_cast<float *>(scratch + 2 * p.E);    // [gate, up, down][E] global scales
+    if (!raw_bytes) raw = nullptr;
     int32_t *ds = p.dstate;
 
-    // Shared memory only before the dependency wait.
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < N1 + N2; s++) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], s < N1 ? WG1 : WG2);
-        }
-        s_abort = 0;
-        fence_barrier_init();
-    }
-    __syncthreads();
     // Everything this layer reads may come from the previous kernel in the stream.
     grid_dep_wait();
-    if (threadIdx.x == 0) DEC_MARK(0);
 
-    // Consumers: this warp's phase-1 activations first, so their loads are in
-    // flight while the CTA routes.
-    const int wi1 = warp % WG1, g1 = warp / WG1;
-    uint4 bx[kMaxRW][4];
-    if (warp < kDecCW) {
-#pragma unroll
-        for (int kk = 0; kk < kMaxRW; kk++) {
-            const int k0 = 128 * (wi1 + kk * WG1) + 32 * q;
-            if (gq < T && k0 < H) {
-                load_x32(p, gq, k0, bx[kk]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 4; i++) bx[kk][i] = make_uint4(0, 0, 0, 0);
-            }
+    // While warps 0..T-1 route, warps 8..15 stage the activations: per-token amax
+    // -> power-of-two shift -> F16 in shared memory (token slots past T and
+    // columns past H zero), and fetch every expert's three global scales.
+    const bool int8 = p.act_type == NVFP4_MOE_ACT_INT8;
+    auto stage = [&]() {
+        const int st = threadIdx.x - kSlots * 32, sw = st >> 5, nst = kDecThreads - kSlots * 32;
+        for (int c = st; c < raw_bytes / 16; c += nst)
+            cp_async16(raw + 16 * c, static_cast<const uint8_t *>(p.act) + 16 * c);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        for (int e = st; e < p.E; e += nst) {
+            gsc[e] = p.gate_global[e];
+            gsc[p.E + e] = p.up_global[e];
+            gsc[2 * p.E + e] = p.down_global[e];
         }
-    }
-
-    // routing scratch: the partial-sum buffers, unused until phase 1
-    cta_route<NPER>(p, R, blockIdx.x == 0, reinterpret_cast<int *>(dsm),
-                    reinterpret_cast<int *>(dsm) + 1024);
-    if (threadIdx.x == 0) DEC_MARK(1);
-    const int U = R.U;
-    const int per1 = I / 8, per2 = H / 16;        // items per used expert
-    const int n1 = U * per1, n2 = U * per2;
-    const int G = gridDim.x, c = blockIdx.x;
-    const int a1 = (int)((long long)n1 * c / G), b1 = (int)((long long)n1 * (c + 1) / G);
-    const int a2 = (int)((long long)n2 * c / G), b2 = (int)((long long)n2 * (c + 1) / G);
-
-    if (warp >= kDecCW) {
-        // ----------------------------------------------------------- producers
-        // One lane of the first producer warp fills ring A with this CTA's
-        // phase-1 items, one lane of the second ring B with its phase-2 items,
-        // each as fast as slots free up (separate warps: neither spin-wait can
-        // hold the other back).
-        if (lane == 0) {
-            const bool A = warp == kDecCW;
-            const int n = A ? b1 - a1 : b2 - a2, N = A ? N1 : N2, S = A ? S1 : S2;
-            uint8_t *ring = A ? ringA : ringB;
-            uint64_t *fb = A ? full : full + N1, *eb = A ? empty : empty + N1;
-            int k = 0;
-            for (; k < n; k++) {
-                const int slot = k % N;
-                if (k >= N && !mbar_wait(&eb[slot], ((k / N) - 1) & 1, abort, p.status, 120, kDecWaitNs))
-                    break;
-                uint8_t *dst = ring + (size_t)slot * S;
-                mbar_arrive_expect_tx(&fb[slot], S);
-                if (A) {
-                    const int gi = a1 + k, u = gi / per1, m0 = (gi - u * per1) * 8;
-                    const size_t row = (size_t)R.uniq[u] * I + m0;
-                    bulk_g2s(dst, p.gate_codes + row * (H / 2), 4 * H, &fb[slot]);
-                    bulk_g2s(dst + 4 * H, p.up_codes + row * (H / 2), 4 * H, &fb[slot]);
-                    bulk_g2s(dst + 8 * H, p.gate_scales + row * (H / 16), H / 2, &fb[slot]);
-                    bulk_g2s(dst + 8 * H + H / 2, p.up_scales + row * (H / 16), H / 2, &fb[slot]);
-                } else {
-                    const int gi = a2 + k, u = gi / per2, r0 = (gi - u * per2) * 16;
-                    const size_t row = (size_t)R.uniq[u] * H + r0;
-                    bulk_g2s(dst, p.down_codes + row * (I / 2), 8 * I, &fb[slot]);
-                    bulk_g2s(dst + 8 * I, p.down_scales + row * (I / 16), I, &fb[slot]);
-                }
-            }
-            // The last fill of every slot must have landed before the CTA exits
-            // (the consumers normally waited for each; not after an abort).
-            for (int j = k - 1; j >= 0 && j >= k - N; j--)
-                mbar_wait_drain(&fb[j % N], (j / N) & 1, kDecDrainNs);
+        const int h8 = H / 8, p8 = ld1 / 8;
+        for (int c = st; c < kSlots * (p8 - h8) + (kSlots - T) * h8; c += nst) {
+            int t, k8;
+            if (c < kSlots * (p8 - h8)) { t = c / (p8 - h8); k8 = h8 + c % (p8 - h8); }
+            else { const int d = c - kSlots * (p8 - h8); t = T + d / h8; k8 = d % h8; }
+            uint2 *dst = reinterpret_cast<uint2 *>(xs + (size_t)t * ld1 + 8 * k8);
+            dst[0] = make_uint2(0, 0);
+            if (8 * k8 + 4 < ld1) dst[1] = make_uint2(0, 0);
         }
-    } else {
-        // ------------------------------------------------------ consumers
-        // Per-token activation amax (this warp's rounds; every K round is covered
-        // by every group), then the F16 B fragments.
-        const bool int8 = p.act_type == NVFP4_MOE_ACT_INT8;
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"r"(nst) : "memory");
         if (!int8) {
-            float m = 0.0f;
+            for (int t = sw; t < T; t += nst / 32) {
+                float m = 0.0f;
+                for (int k8 = lane; k8 < h8; k8 += 32) {
+                    float v[8];
+                    act8(p, raw, t, k8, v);
 #pragma unroll
-            for (int kk = 0; kk < kMaxRW; kk++) m = fmaxf(m, raw_amax(bx[kk]));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-            if (q == 0 && gq < T) atomicMax(&R.amax[gq], __float_as_uint(m));
-        }
-        named_bar(kBarConsumers, kDecCW * 32);
-        if (threadIdx.x == 0) DEC_MARK(2);
-        {
-            const int sh = (int8 || gq >= T) ? 0 : pow2_shift_for(__uint_as_float(R.amax[gq]));
-#pragma unroll
-            for (int kk = 0; kk < kMaxRW; kk++) to_f16_frags(int8, sh, bx[kk]);
-        }
-
-        // ------------------------------------------- phase 1: gate/up + SwiGLU
-        // A group of WG1 warps takes every groups1-th item of the CTA's range.
-        // Each item's partial sums are reduced one iteration later by one warp of
-        // the group (rotating), so that work overlaps the next item's MMAs.
-        {
-            const int groups1 = kDecCW / WG1, n1c = b1 - a1, w0 = g1 * WG1;
-            const int nmine = n1c > g1 ? cdiv(n1c - g1, groups1) : 0;
-            for (int it = 0; it <= nmine; it++) {
-                const int k = g1 + it * groups1;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                if (it < nmine) {
-                    const int slot = k % N1;
-                    const bool got = warp_wait(&full[slot], (k / N1) & 1, abort, p.status, 121);
-                    if (threadIdx.x == 0 && it == 0) DEC_MARK(3);
-                    if (got) {
-                        const uint8_t *base = ringA + (size_t)slot * S1;
-#pragma unroll
-                        for (int kk = 0; kk < kMaxRW; kk++) {
-                            const int r = wi1 + kk * WG1;
-                            if (r < NR1) {
-                                uint4 ca, cb;
-                                uint32_t sa, sb;
-                                // rows 0..7 of the slot are gate rows, 8..15 the matching up rows
-                                slot_round(base, H / 2, gq, gq + 8, r, q, ca, cb, sa, sb);
-                                round_mma(acc, ca, cb, sa, sb, bx[kk]);
-                            }
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[slot]);
+                    for (int j = 0; j < 8; j++) m = fmaxf(m, fabsf(v[j]));
                 }
-                if (it > 0 && wi1 == (it - 1) % WG1) {
-                    // item it - 1: the lane holds gate (x, y) and up (z, w) of
-                    // intermediate m0 + gq for tokens 2q, 2q + 1
-                    const float4 s = group_sum(part, w0, WG1, (it - 1) & 1, lane);
-                    const int gi = a1 + k - groups1, u = gi / per1, m0 = (gi - u * per1) * 8;
-                    const int e = R.uniq[u];
-                    const float sg = __ldg(p.gate_global + e), su = __ldg(p.up_global + e);
-                    bool fin = true;
 #pragma unroll
-                    for (int cc = 0; cc < 2; cc++) {
-                        const int tok = 2 * q + cc;
-                        const int pos = tok < T ? R.upos[u * kSlots + tok] : -1;
-                        if (pos >= 0) {
-                            const float xs = token_xscale(p, R, tok);
-                            const float gv = (cc ? s.y : s.x) * sg * xs, uv = (cc ? s.w : s.z) * su * xs;
-                            const float hf = silu(gv) * uv * exp2i(token_hexp(p, R, tok));
-                            fin &= fits_f16(hf);
-                            p.h[(size_t)pos * I + m0 + gq] = __float2half_rn(hf);
-                        }
-                    }
-                    if (!fin) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, kNfH | e);
-                    __syncwarp();
-                    if (lane == 0) red_release_add(ds + kDsReady + u, 1);
-                }
-                if (it < nmine)
-                    part[((size_t)warp * 2 + (it & 1)) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-                named_bar(1 + g1, WG1 * 32);
+                for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (lane == 0) R.amax[t] = __float_as_uint(m);
             }
         }
-
-        // ------------------------------------------------ phase 2: down rows
-        named_bar(kBarConsumers, kDecCW * 32);   // named barrier ids are reused below
-        if (threadIdx.x == 0) DEC_MARK(4);
-        {
-            const int wi2 = warp % WG2, g2 = warp / WG2, w0 = g2 * WG2;
-            const int groups2 = kDecCW / WG2, n2c = b2 - a2;
-            const int nmine = n2c > g2 ? cdiv(n2c - g2, groups2) : 0;
-            int cur_u = -1;
-            for (int it = 0; it <= nmine; it++) {
-                const int k = g2 + it * groups2;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                if (it < nmine) {
-                    const int gi = a2 + k, u = gi / per2;
-                    if (u != cur_u) {
-                        // this expert's h rows, once all its phase-1 items are done
-                        int ok = 1;
-                        if (lane == 0) ok = wait_geq(ds + kDsReady + u, per1, p.status, 102);
-                        ok = __shfl_sync(0xffffffffu, ok, 0);
-                        if (!ok) *abort = 1;
-                        const int pos = gq < T ? R.upos[u * kSlots + gq] : -1;
-#pragma unroll
-                        for (int kk = 0; kk < kMaxRW; kk++) {
-                            const int k0 = 128 * (wi2 + kk * WG2) + 32 * q;
-                            if (pos >= 0 && k0 < I) {
-                                const uint4 *s = reinterpret_cast<const uint4 *>(p.h + (size_t)pos * I + k0);
-#pragma unroll
-                                for (int i = 0; i < 4; i++) bx[kk][i] = __ldcg(s + i);
-                            } else {
-#pragma unroll
-                                for (int i = 0; i < 4; i++) bx[kk][i] = make_uint4(0, 0, 0, 0);
-                            }
-                        }
-                        cur_u = u;
-                        if (threadIdx.x == 0 && it == 0) DEC_MARK(5);
-                    }
-                    const int slot = k % N2;
-                    if (warp_wait(&full[N1 + slot], (k / N2) & 1, abort, p.status, 122)) {
-                        const uint8_t *base = ringB + (size_t)slot * S2;
-#pragma unroll
-                        for (int kk = 0; kk < kMaxRW; kk++) {
-                            const int r = wi2 + kk * WG2;
-                            if (r < NR2) {
-                                uint4 ca, cb;
-                                uint32_t sa, sb;
-                                slot_round(base, I / 2, gq, gq + 8, r, q, ca, cb, sa, sb);
-                                round_mma(acc, ca, cb, sa, sb, bx[kk]);
-                            }
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[N1 + slot]);
-                }
-                if (it > 0 && wi2 == (it - 1) % WG2) {
-                    // item it - 1: w * s_d * y of hidden rows r0 + gq (x, y) and
-                    // r0 + gq + 8 (z, w), tokens 2q and 2q + 1, into the pairs' FP32
-                    // rows (h was stored times 2^hexp; undone here)
-                    const float4 s = group_sum(part, w0, WG2, (it - 1) & 1, lane);
-                    const int gi = a2 + k - groups2, u = gi / per2, r0 = (gi - u * per2) * 16;
-                    const int e = R.uniq[u];
-                    const float sd = __ldg(p.down_global + e);
-                    bool fin = true;
-#pragma unroll
-                    for (int cc = 0; cc < 2; cc++) {
-                        const int tok = 2 * q + cc;
-                        const int pos = tok < T ? R.upos[u * kSlots + tok] : -1;
-                        if (pos >= 0) {
-                            const float w = R.uw[u * kSlots + tok] * sd * exp2i(-token_hexp(p, R, tok));
-                            const float y0 = (cc ? s.y : s.x) * w, y1 = (cc ? s.w : s.z) * w;
-                            fin &= isfinite(y0) && isfinite(y1);
-                            p.ybuf[(size_t)pos * H + r0 + gq] = y0;
-                            p.ybuf[(size_t)pos * H + r0 + gq + 8] = y1;
-                        }
-                    }
-                    if (!fin) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, kNfY | e);
-                }
-                if (it < nmine)
-                    part[((size_t)warp * 2 + (it & 1)) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-                named_bar(1 + g2, WG2 * 32);
-            }
+        asm volatile("bar.sync 1, %0;" ::"r"(nst) : "memory");
+        for (int c = st; c < T * h8; c += nst) {
+            const int t = c / h8, k8 = c - t * h8;
+            const int sh = int8 ? 0 : pow2_shift_for(__uint_as_float(R.amax[t]));
+            float v[8];
+            act8(p, raw, t, k8, v);
+            const uint4 pk = pack8_f16(v, sh);
+            uint2 *dst = reinterpret_cast<uint2 *>(xs + (size_t)t * ld1 + 8 * k8);
+            dst[0] = make_uint2(pk.x, pk.y);
+            dst[1] = make_uint2(pk.z, pk.w);
         }
-
-        // ------------------------------------------ weighted combine into out
-        // Once every CTA's down rows are written (which also means every CTA has
-        // read the activations, which out may alias), each CTA adds up its share
-        // of the hidden rows: out_t (+)= sum_j rows(t, j), in order j = 0..K-1.
-        named_bar(kBarConsumers, kDecCW * 32);
-        if (threadIdx.x == 0) {
-            if (!((p.test_flags & NVFP4_MOE_TEST_DECODE_STALL) && blockIdx.x == 0))
-                red_release_add(ds + kDsDone, 1);
-            DEC_MARK(5 + 1);
-            s_ok = wait_geq(ds + kDsDone, G, p.status, 101);
+        if (st < T) {
+            const float am = int8 ? 127.0f * p.act_scale[st] : __uint_as_float(R.amax[st]);
+            R.xsc[st] = int8 ? p.act_scale[st] : exp2i(-pow2_shift_for(am));
+            R.hexp[st] = h_exp_for(am);
         }
-        named_bar(kBarConsumers, kDecCW * 32);
-        if (s_ok) {
-            const int rlo = (int)((long long)H * c / G), rhi = (int)((long long)H * (c + 1) / G);
-            const int nrow = rhi - rlo;
-            bool fo = true;
-            for (int o = threadIdx.x; o < nrow * T; o += kDecCW * 32) {
-                const int t = o / nrow, row = rlo + (o - t * nrow);
-                float y[NVFP4_MOE_MAX_TOPK];
+    };
+    cta_route<NPER>(p, R, blockIdx.x == 0, scratch, scratch + p.E, stage);
+    const int U = R.U;
+    const int n8 = U * (I / 8);
+    const int gb = (int)((long long)n8 * blockIdx.x / gridDim.x);
+    const int ge = (int)((long long)n8 * (blockIdx.x + 1) / gridDim.x);
+    if (threadIdx.x == 0) {
+        P.gb = gb;
+        P.ge = ge;
+    }
+
+    // this warp's gate/up share; its first loads go out before the activations
+    // are staged
+    const int R1 = cdiv(H, 128), R2 = cdiv(I, 128);
+    const int n1 = (ge - gb) * R1;
+    int a1, b1;
+    share(n1, warp, kDecWarps, a1, b1);
+    int x1 = a1;
+    Chunk cur = take_chunk(x1, b1, R1);
+    GuBuf buf0, buf1;
+    {
+        const DecPlan Pl{gb, ge, 0, 0};
+        gu_issue(p, R, Pl, cur, g, q, buf0);
+    }
+
+    __syncthreads();   // P is read by every warp from here on
+
+    // gate/up + SwiGLU: a granule whole in this warp goes to h from registers; a
+    // split one leaves its part in part1 (slot 0: the warp's first granule,
+    // slot 1: its last)
+    int bad1 = -1;   // expert of a non-finite value this thread saw
+    {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        int seg_r0 = cur.r0;
+        const int first_item = a1 / R1;
+        const __half *xrow = xs + g * ld1 + 32 * q;
+        auto step = [&](GuBuf &b, GuBuf &nb) {
+            const Chunk nxt = take_chunk(x1, b1, R1);
+            gu_issue(p, R, P, nxt, g, q, nb);
 #pragma unroll
-                for (int j = 0; j < NVFP4_MOE_MAX_TOPK; j++)
-                    y[j] = j < K ? __ldcg(p.ybuf + (size_t)R.pos[t * K + j] * H + row) : 0.0f;
-                float sum = 0.0f;
-#pragma unroll
-                for (int j = 0; j < NVFP4_MOE_MAX_TOPK; j++)
-                    if (j < K) sum += y[j];
-                float *op = p.out + (size_t)t * H + row;
-                const float v = p.out_add ? *op + sum : sum;
-                fo &= isfinite(v);
-                *op = v;
+            for (int j = 0; j < kGuRounds; j++) {
+                const int r = cur.r0 + j;
+                if (r < cur.r1) {
+                    const __half *xr = xrow + 128 * r;
+                    round_mma(acc, b.ca[j], b.cb[j], b.s[j] & 0xFFFF, b.s[j] >> 16,
+                              [&](int s, uint32_t &v0, uint32_t &v1) {
+                                  const uint2 v = *reinterpret_cast<const uint2 *>(xr + 4 * s);
+                                  v0 = v.x;
+                                  v1 = v.y;
+                              });
+                }
             }
-            if (!fo) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, kNfOut | rlo);
+            if (nxt.r1 == 0 || nxt.item != cur.item) {
+                const float4 v = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                if (cur.r1 - seg_r0 == R1)
+                    swiglu_store(p, R, P, gsc, cur.item, v, g, q, bad1);
+                else
+                    part1[(warp * 2 + (cur.item == first_item ? 0 : 1)) * 32 + lane] = v;
+#pragma unroll
+                for (int c = 0; c < 4; c++) acc[c] = 0.0f;
+                seg_r0 = nxt.r0;
+            }
+            cur = nxt;
+        };
+        while (cur.r1 > 0) {
+            step(buf0, buf1);
+            if (cur.r1 == 0) break;
+            step(buf1, buf0);
         }
     }
 
+    // this CTA's down share: whole 16-row blocks of out, every used expert; the
+    // warp's first loads go out before the barriers
+    int rb0, rb1;
+    share(H / 16, blockIdx.x, gridDim.x, rb0, rb1);
+    const int n2 = (rb1 - rb0) * U * R2;
+    int a2, b2;
+    share(n2, warp, kDecWarps, a2, b2);
+    DnBuf d0, d1;
+    dn_issue(p, R, rb0, dn_cur(a2, U, R2), min(kDnUnits, b2 - a2), g, q, d0);
     __syncthreads();
+    // granules split between warps: their parts summed in warp order
+    for (int j = warp; j < ge - gb; j += kDecWarps) {
+        const int w0 = owner(n1, kDecWarps, j * R1), w1 = owner(n1, kDecWarps, j * R1 + R1 - 1);
+        if (w0 == w1) continue;   // whole in one warp: already stored
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int w = w0; w <= w1; w++) {
+            int wa, wb;
+            share(n1, w, kDecWarps, wa, wb);
+            if (wa == wb) continue;
+            const float4 v = part1[(w * 2 + (j == wa / R1 ? 0 : 1)) * 32 + lane];
+            s.x += v.x;
+            s.y += v.y;
+            s.z += v.z;
+            s.w += v.w;
+        }
+        swiglu_store(p, R, P, gsc, j, s, g, q, bad1);
+    }
+    warp_report(p, bad1, kNfH);
+    // per (used expert, token slot): w * s_d * 2^-hexp (0 where the token did not
+    // choose the expert)
+    for (int k = threadIdx.x; k < U * kSlots; k += blockDim.x) {
+        const int u = k / kSlots, slot = k - u * kSlots;
+        const int pos = slot < T ? R.upos[k] : -1;
+        R.dw[k] = pos >= 0 ? R.uw[k] * gsc[2 * p.E + R.uniq[u]] * exp2i(-R.hexp[slot]) : 0.0f;
+    }
+
+    // grid barrier: every CTA's h is stored (and every CTA has read the
+    // activations: out may alias them)
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (!((p.test_flags & NVFP4_MOE_TEST_DECODE_STALL) && blockIdx.x == 0)) atomicAdd(ds + kDsArrive, 1);
+        P.ok = wait_geq(ds + kDsArrive, gridDim.x, p.status, 101);
+        __threadfence();
+    }
+    __syncthreads();
+    if (P.ok && n2 > 0) {
+        // every pair's h row, K past I zero, then a zero row for absent tokens
+        const int per_row = ld2 / 8, P2 = T * p.K;   // 16-byte pieces per row; pairs
+        for (int c = threadIdx.x; c < (P2 + 1) * per_row; c += blockDim.x) {
+            const int r = c / per_row, k = c - r * per_row;
+            __half *dst = hs + (size_t)r * ld2 + 8 * k;
+            if (r < P2 && 8 * k < I) cp_async16(dst, p.h + (size_t)r * I + 8 * k);
+            else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+        }
+        asm volatile("cp.async.commit_group;\n cp.async.wait_all;" ::: "memory");
+    }
+    __syncthreads();
+
+    // down + weighted combine, in registers: per (row block, expert) the K rounds
+    // sum in acc, then oacc += acc * w * s_d; a row block whole in this warp is
+    // stored from registers, a split one leaves its part in part2
+    int bad2 = -1;
+    if (P.ok) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f}, oacc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int first_rb = a2 / (U * R2);
+        int seg0 = a2;   // first unit of the current row block's part in this warp
+        int x = a2;
+        DnCur cc = dn_cur(a2, U, R2);   // compute cursor: unit x
+        auto step = [&](DnBuf &b, DnBuf &nb) {
+            const int xn = x + kDnUnits;
+            if (xn < b2) {
+                DnCur ic = cc;   // the next chunk starts kDnUnits units on
+#pragma unroll
+                for (int j = 0; j < kDnUnits; j++) dn_next(ic, U, R2);
+                dn_issue(p, R, rb0, ic, min(kDnUnits, b2 - xn), g, q, nb);
+            }
+#pragma unroll
+            for (int j = 0; j < kDnUnits; j++) {
+                const int xx = x + j;
+                if (xx < b2) {
+                    const int rbl = cc.rbl, u = cc.u, r = cc.r;
+                    dn_next(cc, U, R2);
+                    const int pos = g < T ? R.upos[u * kSlots + g] : -1;
+                    const __half *hr = hs + (size_t)(pos >= 0 ? pos : T * p.K) * ld2 + 128 * r + 32 * q;
+                    round_mma(acc, b.ca[j], b.cb[j], b.s[j] & 0xFFFF, b.s[j] >> 16,
+                              [&](int s, uint32_t &v0, uint32_t &v1) {
+                                  const uint2 v = *reinterpret_cast<const uint2 *>(hr + 4 * s);
+                                  v0 = v.x;
+                                  v1 = v.y;
+                              });
+                    const bool last_unit = xx + 1 == b2;
+                    if (r == R2 - 1 || last_unit) {   // expert u done for this row block
+                        const float w0 = R.dw[u * kSlots + 2 * q], w1 = R.dw[u * kSlots + 2 * q + 1];
+                        oacc[0] += acc[0] * w0;
+                        oacc[1] += acc[1] * w1;
+                        oacc[2] += acc[2] * w0;
+                        oacc[3] += acc[3] * w1;
+#pragma unroll
+                        for (int c = 0; c < 4; c++) acc[c] = 0.0f;
+                        if (u == U - 1 || last_unit) {   // row block done in this warp
+                            const float4 o4 = make_float4(oacc[0], oacc[1], oacc[2], oacc[3]);
+                            const bool whole = seg0 == rbl * U * R2 && (r == R2 - 1 && u == U - 1);
+                            if (whole)
+                                store_out(p, rb0 + rbl, o4, g, q, bad2);
+                            else
+                                part2[(warp * 2 + (rbl == first_rb ? 0 : 1)) * 32 + lane] = o4;
+#pragma unroll
+                            for (int c = 0; c < 4; c++) oacc[c] = 0.0f;
+                            seg0 = xx + 1;
+                        }
+                    }
+                }
+            }
+            x = xn;
+        };
+        while (x < b2) {
+            step(d0, d1);
+            if (x >= b2) break;
+            step(d1, d0);
+        }
+    }
+    __syncthreads();
+    // row blocks split between warps: their parts summed in warp order
+    if (P.ok) {
+        const int per_rb = U * R2;
+        for (int rbl = warp; rbl < rb1 - rb0; rbl += kDecWarps) {
+            const int w0 = owner(n2, kDecWarps, rbl * per_rb), w1 = owner(n2, kDecWarps, rbl * per_rb + per_rb - 1);
+            if (w0 == w1) continue;   // whole in one warp: already stored
+            float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int w = w0; w <= w1; w++) {
+                int wa, wb;
+                share(n2, w, kDecWarps, wa, wb);
+                if (wa == wb) continue;
+                const float4 v = part2[(w * 2 + (rbl == wa / per_rb ? 0 : 1)) * 32 + lane];
+                s.x += v.x;
+                s.y += v.y;
+                s.z += v.z;
+                s.w += v.w;
+            }
+            store_out(p, rb0 + rbl, s, g, q, bad2);
+        }
+    }
+    warp_report(p, bad2, kNfOut);
+
     if (blockIdx.x == 0) publish_route(p, R);
     // The last CTA done resets the counters for the next launch.
     if (threadIdx.x == 0) {
         __threadfence();
-        if (atomicAdd(ds + kDsExit, 1) == G - 1) {
-            for (int u = 0; u < U; u++) ds[kDsReady + u] = 0;
-            ds[kDsDone] = 0;
+        if (atomicAdd(ds + kDsExit, 1) == (int)gridDim.x - 1) {
+            ds[kDsArrive] = 0;
             ds[kDsExit] = 0;
             __threadfence();
         }
-        DEC_MARK(7);
     }
     // The next layer's grid may launch once every CTA is here.
     grid_dep_launch();
 }
-
-#ifdef NVMOE_DEC_TRACE
-}  // namespace nvmoe
-extern "C" NVFP4_MOE_API int nvfp4_moe_dbg_trace(unsigned long long *host, int n) {
-    return (int)cudaMemcpyFromSymbol(host, nvmoe::g_dec_trace, sizeof(unsigned long long) * n);
-}
-namespace nvmoe {
-#endif
 
 int sm_count() {
     int dev = 0, sms = 148;
@@ -703,34 +758,42 @@ int sm_count() {
 
 int decode_grid() { return sm_count(); }
 
-// Ring slots: about half the budget for phase-1 items (at most 8), the rest for
-// phase-2 items (at most 32).
-static void decode_plan(int H, int I, int &n1, int &n2) {
-    const int avail = kDecSmemBudget - kPartBytes - 16 * (8 + 32);   // barriers at most
-    const int s1 = 9 * H, s2 = 9 * I;
-    n1 = min(8, max(2, avail / 2 / s1));
-    n2 = min(32, (avail - n1 * s1) / s2);
+// Dynamic shared memory: the gate/up phase's storage (F16 activation tile, raw
+// activations when they fit, split-granule parts) and the down phase's (every
+// pair's h row, split-row-block parts) share one region; the routing scratch
+// and every expert's three global scales follow. Kept well below the SM's 256 KB: L1 and shared memory share that
+// storage, and the weight loads in flight need L1 room (a kernel holding over
+// 200 KB of shared memory streamed about half as fast).
+constexpr size_t kDecSmemMax = 150 * 1024;
+constexpr size_t kPartBytes = (size_t)kDecWarps * 2 * 32 * 16;
+
+static size_t decode_union_for(int T, int K, int H, int I, int act_type, bool raw) {
+    const size_t ph1 = (size_t)kSlots * dec_ld1(H) * 2 + (raw ? (size_t)T * raw_act_bytes(act_type, H) : 0) +
+                       kPartBytes;
+    const size_t ph2 = (size_t)(T * K + 1) * dec_ld2(I) * 2 + kPartBytes;
+    return ph1 > ph2 ? ph1 : ph2;
+}
+size_t decode_union_bytes(int T, int K, int H, int I, int act_type, bool raw) {
+    return decode_union_for(T, K, H, I, act_type, raw);
+}
+static size_t decode_smem_for(int T, int K, int E, int H, int I, int act_type, bool raw) {
+    return decode_union_for(T, K, H, I, act_type, raw) + (size_t)5 * E * 4;
+}
+bool decode_raw_staged(int T, int K, int E, int H, int I, int act_type) {
+    return decode_smem_for(T, K, E, H, I, act_type, true) <= kDecSmemMax;
 }
 
-bool decode_fits(int H, int I) {
+bool decode_fits(int H, int I, int K, int E) {
     if (H % 32 || I % 32) return false;
-    if (dec_group_warps(cdiv(H, 128)) == 0 || dec_group_warps(cdiv(I, 128)) == 0) return false;
-    int n1, n2;
-    decode_plan(H, I, n1, n2);
-    return n2 >= 2 && 2 * 9 * H <= kDecSmemBudget - kPartBytes;
-}
-
-static size_t decode_smem(int H, int I, int n1, int n2) {
-    return (size_t)kPartBytes + (size_t)n1 * 9 * H + (size_t)n2 * 9 * I + 16 * (size_t)(n1 + n2);
+    return decode_smem_for(kSlots, K, E, H, I, NVFP4_MOE_ACT_BF16, false) <= kDecSmemMax;
 }
 
 template <int NPER>
-static cudaError_t launch_layer(Params p, cudaStream_t s) {
-    decode_plan(p.H, p.I, p.dec_n1, p.dec_n2);
+static cudaError_t launch_layer(const Params &p, cudaStream_t s) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(decode_grid());
     cfg.blockDim = dim3(kDecThreads);
-    cfg.dynamicSmemBytes = decode_smem(p.H, p.I, p.dec_n1, p.dec_n2);
+    cfg.dynamicSmemBytes = decode_smem_for(p.T, p.K, p.E, p.H, p.I, p.act_type, p.dec_raw);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -751,8 +814,8 @@ cudaError_t launch_decode(const Params &p, cudaStream_t s) {
 }
 
 cudaError_t decode_init() {
-    // dynamic shared memory above the 48 KB default: the rings take most of the SM
-    const int big = kDecSmemBudget;
+    // dynamic shared memory above the 48 KB default (the activations grow with H)
+    const int big = (int)kDecSmemMax;
     const cudaError_t r[] = {
         cudaFuncSetAttribute(decode_layer_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
         cudaFuncSetAttribute(decode_layer_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),

@@ -100,12 +100,12 @@ inline bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 
 
 // Whether a call with T tokens takes the decode kernel (else the grouped GEMMs).
 bool use_decode(const nvfp4_moe_dims &d, int T) {
-    return T <= NVFP4_MOE_DECODE_MAX_T && decode_fits(d.hidden, d.inter);
+    return T <= NVFP4_MOE_DECODE_MAX_T && decode_fits(d.hidden, d.inter, d.top_k, d.n_experts);
 }
 
 struct WsLayout {
     size_t cnt, ids, wts, hist, cbase, counts, offsets, perm, inv, ptok, pw, ps, xscale, ph, phinv, tiles_gu,
-        tiles_dn, ybuf, xh, h, total;
+        tiles_dn, xh, h, total;
     int nch, max_gu, max_dn;
 };
 
@@ -141,7 +141,6 @@ WsLayout layout(const nvfp4_moe_dims &d, int T) {
     L.phinv = take(decode ? 0 : (size_t)T * 4);
     L.tiles_gu = take((size_t)L.max_gu * sizeof(Tile));
     L.tiles_dn = take((size_t)L.max_dn * sizeof(Tile));
-    L.ybuf = take(decode ? P * d.hidden * 4 : 0);   // decode: FP32 down rows per pair
     L.xh = take(decode ? 0 : P * d.hidden * 2);   // decode stages activations in shared memory
     L.h = take(P * d.inter * 2);
     L.total = o;
@@ -306,7 +305,6 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     p.phinv = reinterpret_cast<float *>(b + L.phinv);
     p.tiles_gu = reinterpret_cast<Tile *>(b + L.tiles_gu);
     p.tiles_dn = reinterpret_cast<Tile *>(b + L.tiles_dn);
-    p.ybuf = reinterpret_cast<float *>(b + L.ybuf);
     p.xh = reinterpret_cast<__half *>(b + L.xh);
     p.h = reinterpret_cast<__half *>(b + L.h);
     p.status = h->status;
@@ -323,6 +321,8 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     if (decode) {
         if (!h->dstate) return NVFP4_MOE_ERR_INVALID_ARG;
         p.dstate = reinterpret_cast<int32_t *>(h->dstate);
+        p.dec_raw = decode_raw_staged(T, d.top_k, d.n_experts, d.hidden, d.inter, io->act_type) ? 1 : 0;
+        p.dec_union = (int32_t)decode_union_bytes(T, d.top_k, d.hidden, d.inter, io->act_type, p.dec_raw);
     }
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -428,7 +428,7 @@ void nvfp4_moe_destroy(nvfp4_moe_t *h) {
 // library holds until the process exits.
 namespace {
 
-constexpr size_t kStaticScratchBytes = size_t(2) << 20;  // 2 MiB per device
+constexpr size_t kStaticScratchBytes = size_t(1) << 20;  // 1 MiB per device
 constexpr size_t kStaticStatusBytes = 256;               // status words, then decode state, workspace
 constexpr int kMaxDevices = 64;
 
