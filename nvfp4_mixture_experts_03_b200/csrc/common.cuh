@@ -30,9 +30,10 @@ enum : int { kStatusCode = 0, kStatusDetail = 1, kStatusWords = 64 };
 
 // Per-call routing/tile counters kept in the workspace (int32 words).
 enum : int { kCntTilesGu = 0, kCntTilesDn = 1, kCntUniq = 2, kCntWords = 64 };
-// Decode state (per handle, int32 counters, zero between launches): kDsArrive:
-// CTAs past the gate/up phase (the grid barrier); kDsExit: CTAs done.
-enum : int { kDsArrive = 0, kDsExit = 1, kDsInts = 64 };
+// Decode state (per handle, int32 counters): kDsArrive: CTAs at the grid barrier
+// (zero between launches); kDsGen: barrier generation (counts launches; any
+// value is valid, so the state may be cleared at any time between launches).
+enum : int { kDsArrive = 0, kDsGen = 1, kDsInts = 64 };
 inline size_t decode_state_bytes() { return (size_t)kDsInts * 4; }
 
 struct Tile {  // one grouped-GEMM tile
@@ -87,7 +88,6 @@ struct Params {
     int32_t max_tiles_gu, max_tiles_dn;
     int32_t *dstate;           // decode: counters (kDs*), zero between launches
     int32_t dec_union;         // decode: bytes of the phase-shared dynamic shared memory
-    int32_t dec_raw;           // decode: raw activations copied to shared memory first
     int32_t test_flags;        // NVFP4_MOE_TEST_* (test hooks; 0 in production)
 };
 
@@ -399,8 +399,7 @@ constexpr int kDecWarpsPerCta = 16;                // warps of a decode CTA
 // Whether the decode kernel's shared-memory plan holds layers of these dims (else
 // small batches take the grouped-GEMM path).
 bool decode_fits(int H, int I, int K, int E);
-size_t decode_union_bytes(int T, int K, int H, int I, int act_type, bool raw);
-bool decode_raw_staged(int T, int K, int E, int H, int I, int act_type);
+size_t decode_union_bytes(int T, int K, int H, int I);
 // mode 0: gate/up + SwiGLU, map_b = F16 activations [P][H]; mode 1: down, map_b =
 // h [P][I]; both 64 x 64 boxes
 // Tensor maps of the packed E2M1 code planes (bytes; 128-byte x 64-row boxes for

@@ -17,7 +17,8 @@
 //     its (granule, 128-wide K round) units evenly over its warps, sums a granule
 //     split between warps in shared memory in warp order, and stores h (F16 with
 //     a per-token power-of-two range exponent) at each pair's position;
-//   one grid barrier (bounded wait): every h is stored, every CTA has read the
+//   one grid barrier (bounded wait; the last CTA to arrive resets the count and
+//     bumps a generation word the others wait on): every h is stored, every CTA has read the
 //     activations (out may alias them);
 //   down + weighted combine: each CTA owns whole 16-row blocks of out and, for
 //     every used expert, streams those rows of the expert's down matrix (whole
@@ -375,39 +376,12 @@ __device__ inline void cp_async16(void *smem, const void *gmem) {
                  : "memory");
 }
 
-// Raw activation bytes per token held in shared memory (0: FP32 input, which is
-// read from global memory instead).
-__host__ __device__ inline int raw_act_bytes(int act_type, int H) {
-    return act_type == NVFP4_MOE_ACT_BF16 ? 2 * H : (act_type == NVFP4_MOE_ACT_INT8 ? H : 0);
-}
-
-// Eight activations of token t (group k8) as FP32, from the shared raw copy when
-// there is one, else from global memory.
-__device__ inline void act8(const Params &p, const uint8_t *raw, int t, int k8, float (&v)[8]) {
-    if (!raw) {
-        load_act8(p, t, k8, v);
-    } else if (p.act_type == NVFP4_MOE_ACT_BF16) {
-        const uint4 u = reinterpret_cast<const uint4 *>(raw + (size_t)t * 2 * p.H)[k8];
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            v[2 * i] = __uint_as_float(w[i] << 16);
-            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-        }
-    } else {
-        const uint2 u = reinterpret_cast<const uint2 *>(raw + (size_t)t * p.H)[k8];
-        const uint32_t w[2] = {u.x, u.y};
-#pragma unroll
-        for (int i = 0; i < 8; i++) v[i] = (float)(int8_t)(w[i >> 2] >> (8 * (i & 3)));
-    }
-}
-
-// Bounded wait until *word >= target (one thread); latches TIMEOUT on give-up.
-__device__ inline bool wait_geq(const int32_t *word, int target, int32_t *status, int where) {
+// Bounded wait until *word != old (one thread); latches TIMEOUT on give-up.
+__device__ inline bool wait_ne(const int32_t *word, int old, int32_t *status, int where) {
     const volatile int32_t *v = word;
-    if (*v >= target) return true;
+    if (*v != old) return true;
     const uint64_t t0 = globaltimer();
-    while (*v < target) {
+    while (*v == old) {
         __nanosleep(32);
         if (globaltimer() - t0 > kDecWaitNs) {
             latch_status(status, NVFP4_MOE_ERR_TIMEOUT, where);
@@ -421,6 +395,10 @@ __device__ inline bool wait_geq(const int32_t *word, int target, int32_t *status
 // the K rounds rounded up, plus a few elements so that rows fall in different
 // banks.
 __host__ __device__ inline int dec_ld1(int H) { return cdiv(H, 128) * 128 + 4; }
+// Bytes of the activation tile, rounded up to 16 (the parts after it are float4).
+__host__ __device__ inline size_t dec_xs_bytes(int T, int H) {
+    return ((size_t)(T + 1) * dec_ld1(H) * 2 + 15) & ~(size_t)15;
+}
 __host__ __device__ inline int dec_ld2(int I) { return cdiv(I, 128) * 128 + 8; }
 
 // [a, b) = worker w's share of n units when W workers split them evenly in
@@ -448,53 +426,49 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     const int H = p.H, I = p.I, T = p.T;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int ld1 = dec_ld1(H), ld2 = dec_ld2(I);
-    const int raw_bytes = p.dec_raw ? T * raw_act_bytes(p.act_type, H) : 0;
-    // gate/up phase: [8][ld1] F16 activations, raw activations, split-granule parts;
+    // gate/up phase: [T + 1][ld1] F16 activations (row T: zeros, for the token
+    // slots past T), split-granule parts;
     // down phase (same storage): [P + 1][ld2] h rows (row P: zeros), split-row-block parts
     __half *xs = reinterpret_cast<__half *>(dsm);
-    uint8_t *raw = reinterpret_cast<uint8_t *>(xs + kSlots * ld1);
-    float4 *part1 = reinterpret_cast<float4 *>(raw + raw_bytes);
+    float4 *part1 = reinterpret_cast<float4 *>(dsm + dec_xs_bytes(T, H));   // 16-byte aligned
     __half *hs = reinterpret_cast<__half *>(dsm);
     float4 *part2 = reinterpret_cast<float4 *>(hs + (size_t)(p.T * p.K + 1) * ld2);
     int *scratch = reinterpret_cast<int *>(dsm + p.dec_union);   // routing: 2E ints
     float *gsc = reinterpret_cast<float *>(scratch + 2 * p.E);    // [gate, up, down][E] global scales
-    if (!raw_bytes) raw = nullptr;
     int32_t *ds = p.dstate;
 
     // Everything this layer reads may come from the previous kernel in the stream.
     grid_dep_wait();
+    // this launch's barrier generation: no CTA can open the next one before every
+    // CTA (this one included) has arrived, hence read it
+    const int gen0 = threadIdx.x == 0 ? *reinterpret_cast<volatile int32_t *>(ds + kDsGen) : 0;
 
     // While warps 0..T-1 route, warps 8..15 stage the activations: per-token amax
-    // -> power-of-two shift -> F16 in shared memory (token slots past T and
-    // columns past H zero), and fetch every expert's three global scales.
+    // -> power-of-two shift -> F16 in shared memory (columns past H and the zero
+    // row T are zero), and fetch every expert's three global scales.
     const bool int8 = p.act_type == NVFP4_MOE_ACT_INT8;
     auto stage = [&]() {
         const int st = threadIdx.x - kSlots * 32, sw = st >> 5, nst = kDecThreads - kSlots * 32;
-        for (int c = st; c < raw_bytes / 16; c += nst)
-            cp_async16(raw + 16 * c, static_cast<const uint8_t *>(p.act) + 16 * c);
-        asm volatile("cp.async.commit_group;" ::: "memory");
         for (int e = st; e < p.E; e += nst) {
             gsc[e] = p.gate_global[e];
             gsc[p.E + e] = p.up_global[e];
             gsc[2 * p.E + e] = p.down_global[e];
         }
         const int h8 = H / 8, p8 = ld1 / 8;
-        for (int c = st; c < kSlots * (p8 - h8) + (kSlots - T) * h8; c += nst) {
+        for (int c = st; c < T * (p8 - h8) + p8; c += nst) {
             int t, k8;
-            if (c < kSlots * (p8 - h8)) { t = c / (p8 - h8); k8 = h8 + c % (p8 - h8); }
-            else { const int d = c - kSlots * (p8 - h8); t = T + d / h8; k8 = d % h8; }
+            if (c < T * (p8 - h8)) { t = c / (p8 - h8); k8 = h8 + c % (p8 - h8); }
+            else { t = T; k8 = c - T * (p8 - h8); }
             uint2 *dst = reinterpret_cast<uint2 *>(xs + (size_t)t * ld1 + 8 * k8);
             dst[0] = make_uint2(0, 0);
             if (8 * k8 + 4 < ld1) dst[1] = make_uint2(0, 0);
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        asm volatile("bar.sync 1, %0;" ::"r"(nst) : "memory");
         if (!int8) {
             for (int t = sw; t < T; t += nst / 32) {
                 float m = 0.0f;
                 for (int k8 = lane; k8 < h8; k8 += 32) {
                     float v[8];
-                    act8(p, raw, t, k8, v);
+                    load_act8(p, t, k8, v);
 #pragma unroll
                     for (int j = 0; j < 8; j++) m = fmaxf(m, fabsf(v[j]));
                 }
@@ -508,7 +482,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
             const int t = c / h8, k8 = c - t * h8;
             const int sh = int8 ? 0 : pow2_shift_for(__uint_as_float(R.amax[t]));
             float v[8];
-            act8(p, raw, t, k8, v);
+            load_act8(p, t, k8, v);
             const uint4 pk = pack8_f16(v, sh);
             uint2 *dst = reinterpret_cast<uint2 *>(xs + (size_t)t * ld1 + 8 * k8);
             dst[0] = make_uint2(pk.x, pk.y);
@@ -554,7 +528,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         int seg_r0 = cur.r0;
         const int first_item = a1 / R1;
-        const __half *xrow = xs + g * ld1 + 32 * q;
+        const __half *xrow = xs + (size_t)(g < T ? g : T) * ld1 + 32 * q;
         auto step = [&](GuBuf &b, GuBuf &nb) {
             const Chunk nxt = take_chunk(x1, b1, R1);
             gu_issue(p, R, P, nxt, g, q, nb);
@@ -631,8 +605,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
-        if (!((p.test_flags & NVFP4_MOE_TEST_DECODE_STALL) && blockIdx.x == 0)) atomicAdd(ds + kDsArrive, 1);
-        P.ok = wait_geq(ds + kDsArrive, gridDim.x, p.status, 101);
+        // the last CTA to arrive resets the count and opens the next generation
+        bool open = false;
+        if (!((p.test_flags & NVFP4_MOE_TEST_DECODE_STALL) && blockIdx.x == 0) &&
+            atomicAdd(ds + kDsArrive, 1) == (int)gridDim.x - 1) {
+            atomicExch(ds + kDsArrive, 0);
+            __threadfence();
+            atomicAdd(ds + kDsGen, 1);
+            open = true;
+        }
+        P.ok = open || wait_ne(ds + kDsGen, gen0, p.status, 101);
         __threadfence();
     }
     __syncthreads();
@@ -736,15 +718,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     warp_report(p, bad2, kNfOut);
 
     if (blockIdx.x == 0) publish_route(p, R);
-    // The last CTA done resets the counters for the next launch.
-    if (threadIdx.x == 0) {
-        __threadfence();
-        if (atomicAdd(ds + kDsExit, 1) == (int)gridDim.x - 1) {
-            ds[kDsArrive] = 0;
-            ds[kDsExit] = 0;
-            __threadfence();
-        }
-    }
     // The next layer's grid may launch once every CTA is here.
     grid_dep_launch();
 }
@@ -758,8 +731,8 @@ int sm_count() {
 
 int decode_grid() { return sm_count(); }
 
-// Dynamic shared memory: the gate/up phase's storage (F16 activation tile, raw
-// activations when they fit, split-granule parts) and the down phase's (every
+// Dynamic shared memory: the gate/up phase's storage (F16 activation tile,
+// split-granule parts) and the down phase's (every
 // pair's h row, split-row-block parts) share one region; the routing scratch
 // and every expert's three global scales follow. Kept well below the SM's 256 KB: L1 and shared memory share that
 // storage, and the weight loads in flight need L1 room (a kernel holding over
@@ -767,25 +740,19 @@ int decode_grid() { return sm_count(); }
 constexpr size_t kDecSmemMax = 150 * 1024;
 constexpr size_t kPartBytes = (size_t)kDecWarps * 2 * 32 * 16;
 
-static size_t decode_union_for(int T, int K, int H, int I, int act_type, bool raw) {
-    const size_t ph1 = (size_t)kSlots * dec_ld1(H) * 2 + (raw ? (size_t)T * raw_act_bytes(act_type, H) : 0) +
-                       kPartBytes;
+static size_t decode_union_for(int T, int K, int H, int I) {
+    const size_t ph1 = dec_xs_bytes(T, H) + kPartBytes;
     const size_t ph2 = (size_t)(T * K + 1) * dec_ld2(I) * 2 + kPartBytes;
     return ph1 > ph2 ? ph1 : ph2;
 }
-size_t decode_union_bytes(int T, int K, int H, int I, int act_type, bool raw) {
-    return decode_union_for(T, K, H, I, act_type, raw);
-}
-static size_t decode_smem_for(int T, int K, int E, int H, int I, int act_type, bool raw) {
-    return decode_union_for(T, K, H, I, act_type, raw) + (size_t)5 * E * 4;
-}
-bool decode_raw_staged(int T, int K, int E, int H, int I, int act_type) {
-    return decode_smem_for(T, K, E, H, I, act_type, true) <= kDecSmemMax;
+size_t decode_union_bytes(int T, int K, int H, int I) { return decode_union_for(T, K, H, I); }
+static size_t decode_smem_for(int T, int K, int E, int H, int I) {
+    return decode_union_for(T, K, H, I) + (size_t)5 * E * 4;
 }
 
 bool decode_fits(int H, int I, int K, int E) {
     if (H % 32 || I % 32) return false;
-    return decode_smem_for(kSlots, K, E, H, I, NVFP4_MOE_ACT_BF16, false) <= kDecSmemMax;
+    return decode_smem_for(kSlots, K, E, H, I) <= kDecSmemMax;
 }
 
 template <int NPER>
@@ -793,7 +760,7 @@ static cudaError_t launch_layer(const Params &p, cudaStream_t s) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(decode_grid());
     cfg.blockDim = dim3(kDecThreads);
-    cfg.dynamicSmemBytes = decode_smem_for(p.T, p.K, p.E, p.H, p.I, p.act_type, p.dec_raw);
+    cfg.dynamicSmemBytes = decode_smem_for(p.T, p.K, p.E, p.H, p.I);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -321,8 +321,7 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     if (decode) {
         if (!h->dstate) return NVFP4_MOE_ERR_INVALID_ARG;
         p.dstate = reinterpret_cast<int32_t *>(h->dstate);
-        p.dec_raw = decode_raw_staged(T, d.top_k, d.n_experts, d.hidden, d.inter, io->act_type) ? 1 : 0;
-        p.dec_union = (int32_t)decode_union_bytes(T, d.top_k, d.hidden, d.inter, io->act_type, p.dec_raw);
+        p.dec_union = (int32_t)decode_union_bytes(T, d.top_k, d.hidden, d.inter);
     }
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
