@@ -66,6 +66,8 @@ def lib():
         _lib.orc_pair_h.restype = C.c_int
         _lib.orc_pair_h.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_float,
                                     C.c_int32, C.c_void_p, C.c_int32]
+        _lib.orc_router.argtypes = [C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
+                                    C.c_void_p]
         _lib.orc_decode_matrix.argtypes = [C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
                                            C.c_float, C.c_void_p]
     return _lib
@@ -119,6 +121,32 @@ def route(logits, K: int):
     w = np.zeros((T, K), np.float64)
     bad = lib().orc_route(C.c_int32(T), C.c_int32(E), C.c_int32(K), _p(l), _p(ids), _p(w))
     return ids, w, bad
+
+
+def router_input(x, x_scale=None) -> np.ndarray:
+    """The router's FP32 input for the layer's activations: BF16 and FP32 values
+    as they are (exact in FP32); int8 codes as the FP32 product q * scale (one
+    correctly rounded multiply), which is what a reader of the scaled
+    activations holds."""
+    a = _np(x)
+    if a.dtype == np.int16:   # BF16 bits
+        return (a.astype(np.uint16).astype(np.uint32) << 16).view(np.float32)
+    if a.dtype == np.int8:
+        s = _np(x_scale).astype(np.float32)
+        return a.astype(np.float32) * s[:, None]
+    return a.astype(np.float32, copy=False)
+
+
+def router(x_f32, w_r_bf16) -> np.ndarray:
+    """FP64 router logits [T][E] = W_r x for FP32 x [T][H] and BF16 W_r [E][H]."""
+    x = np.ascontiguousarray(_np(x_f32).astype(np.float32, copy=False))
+    w = np.ascontiguousarray(_np(w_r_bf16).astype(np.uint16, copy=False))
+    T, H = x.shape
+    E = w.shape[0]
+    assert w.shape[1] == H
+    out = np.zeros((T, E), np.float64)
+    lib().orc_router(C.c_int32(T), C.c_int32(E), C.c_int32(H), _p(x), _p(w), _p(out))
+    return out
 
 
 def check_ids(ids, E: int) -> int:
@@ -215,10 +243,16 @@ def pair_h(layer, x_row, e: int, *, K: int, x_scale: float = 1.0, plant=0) -> np
 
 
 def forward(layer, x, *, K: int, logits=None, ids=None, wts=None, x_scale=None, sample=None,
-            nthreads: int = 0, plant=0):
-    """Route (or take ids/weights as given) and run the layer.
-    -> dict(out, ids, w, counts, offsets, perm, nonfinite)"""
+            nthreads: int = 0, plant=0, router_w=None):
+    """Route (or take ids/weights as given) and run the layer. With `router_w`
+    (BF16 [E][H]) the logits are the router projection of the layer's input,
+    rounded to FP32 for the selection.
+    -> dict(out, ids, w, counts, offsets, perm, nonfinite[, logits64])"""
     E = _np(layer.gate_global).shape[0]
+    logits64 = None
+    if router_w is not None:
+        logits64 = router(router_input(x, x_scale), router_w)
+        logits = logits64.astype(np.float32)
     if logits is not None:
         ids, w, bad = route(logits, K)
     else:
@@ -228,4 +262,7 @@ def forward(layer, x, *, K: int, logits=None, ids=None, wts=None, x_scale=None, 
     counts, offsets, perm = sort(ids, E)
     out = moe(layer, x, ids, w, K=K, x_scale=x_scale, sample=sample, nthreads=nthreads,
               plant=plant)
-    return dict(out=out, ids=ids, w=w, counts=counts, offsets=offsets, perm=perm, nonfinite=bad)
+    res = dict(out=out, ids=ids, w=w, counts=counts, offsets=offsets, perm=perm, nonfinite=bad)
+    if logits64 is not None:
+        res["logits64"] = logits64
+    return res

@@ -267,6 +267,26 @@ int orc_quantize(int32_t n_mat, int32_t rows, int32_t cols, const uint16_t *w_bf
     return 0;
 }
 
+/* ------------------------------------------------------- router projection */
+
+/* Router logits from the layer's input: the projection that the pages keep on
+ * FP32-exact inputs ("Strata NVFP4" README, "How it differs from upstream
+ * Strata": the prompt path's BF16 projections -- router among them -- take
+ * FP32-exact inputs):
+ *   logits[t][e] = sum_k W_r[e][k] * x[t][k]
+ * W_r is BF16, x is FP32 and is never rounded to BF16; every product and every
+ * sum is FP64. */
+void orc_router(int32_t T, int32_t E, int32_t H, const float *x, const uint16_t *w_r,
+                double *logits) {
+    for (int t = 0; t < T; t++)
+        for (int e = 0; e < E; e++) {
+            double s = 0.0;
+            for (int k = 0; k < H; k++)
+                s += orc_bf16(w_r[(size_t)e * H + k]) * (double)x[(size_t)t * H + k];
+            logits[(size_t)t * E + e] = s;
+        }
+}
+
 /* ------------------------------------------------------------------- layer */
 
 static double act_value(int act_type, const void *row, int k) {

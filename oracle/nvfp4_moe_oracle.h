@@ -69,6 +69,11 @@ int orc_quantize(int32_t n_mat, int32_t rows, int32_t cols, const uint16_t *w_bf
 void orc_decode_matrix(int32_t rows, int32_t cols, const uint8_t *codes, const uint8_t *scales,
                        float glob, double *dst);
 
+/* Router projection: logits[t][e] = sum_k bf16(w_r[e][k]) * x[t][k] in FP64, x FP32
+ * [T][H] (never rounded to BF16), w_r BF16 bits [E][H]. */
+void orc_router(int32_t T, int32_t E, int32_t H, const float *x, const uint16_t *w_r,
+                double *logits);
+
 /* The layer. act_type 0: act = BF16 bits [T][H]; 1: act = int8 [T][H] with
  * act_scale [T] (x = q * scale, the scale applied after the dot products).
  * ids [T][K], wts [T][K] (FP64). out [n][H] FP64 for the n tokens listed in

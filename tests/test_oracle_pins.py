@@ -335,3 +335,84 @@ def test_planted_mistake_is_caught_by_brute_force(plant):
     bad = oracle.forward(layer, x, K=2, logits=logits, plant=plant)["out"]
     assert _rel(good, ref) < 1e-12
     assert _rel(bad, ref) > 1e-2, plant
+
+
+# ------------------------------------------------------------ router projection
+# "Strata NVFP4" README, "How it differs from upstream Strata": the router's BF16
+# projection takes FP32-exact inputs.
+
+def _bf16_bits(a):
+    return (np.asarray(a, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_router_one_hot_rows_return_the_fp32_inputs_unrounded():
+    """W_r row e is one-hot at column k_e (BF16 1.0): logit e of token t is x[t][k_e]
+    itself. The inputs carry bits BF16 cannot hold, so rounding x to BF16 before the
+    product (the mistake the pages' reading rules out) fails here."""
+    H, E, T = 96, 7, 3
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    x[:, ::5] = np.float32(1.0) + np.float32(2.0 ** -20)   # not representable in BF16
+    w = np.zeros((E, H), np.uint16)
+    cols = rng.choice(H, E, replace=False)
+    cols[0] = 0                                             # one column hits the 1 + 2^-20 values
+    w[np.arange(E), cols] = 0x3F80
+    got = oracle.router(x, w)
+    assert np.array_equal(got, x[:, cols].astype(np.float64))
+    assert got[0, 0] == 1.0 + 2.0 ** -20
+
+
+def test_router_all_ones_rows_are_exact_row_sums():
+    """W_r of ones: every logit is the exactly rounded sum of the token's inputs."""
+    H, E, T = 128, 3, 4
+    rng = np.random.default_rng(6)
+    x = (rng.standard_normal((T, H)) * 3).astype(np.float32)
+    w = np.full((E, H), 0x3F80, np.uint16)
+    got = oracle.router(x, w)
+    for t in range(T):
+        want = math.fsum(float(v) for v in x[t])
+        assert np.allclose(got[t], want, rtol=1e-13, atol=1e-12)
+
+
+def test_router_matches_dense_fp64_product():
+    """Random BF16 W_r [E][H] (E != H, so a transposed operand cannot pass) against
+    a library FP64 matrix product of the decoded values."""
+    T, E, H = 5, 24, 160
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    wb = _bf16_bits(rng.standard_normal((E, H)) * 0.05)
+    wf = (wb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    want = x.astype(np.float64) @ wf.T
+    got = oracle.router(x, wb)
+    assert got.shape == (T, E)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-13)
+
+
+def test_router_input_per_activation_type():
+    """BF16 activations reach the router exactly; int8 codes as the FP32 product
+    q * scale, one correctly rounded multiply."""
+    rng = np.random.default_rng(8)
+    xb = torch.from_numpy(rng.standard_normal((2, 64)).astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(oracle.router_input(xb), xb.float().numpy())
+    q = torch.from_numpy(rng.integers(-127, 128, (2, 64)).astype(np.int8))
+    s = torch.tensor([0.0123, 3.7], dtype=torch.float32)
+    want = np.array([[float(np.float32(float(q[t, k]) * float(s[t]))) for k in range(64)]
+                     for t in range(2)], np.float32)
+    assert np.array_equal(oracle.router_input(q, s), want)
+
+
+def test_router_logits_with_k_equal_e_route_to_the_full_softmax():
+    """K = E: the routing weights of the router's logits are the softmax over all
+    experts of those logits (rounded to FP32 for the selection)."""
+    T, E, H = 3, 6, 64
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    wb = _bf16_bits(rng.standard_normal((E, H)) * 0.1)
+    l32 = oracle.router(x, wb).astype(np.float32).astype(np.float64)
+    ids, w, bad = oracle.route(l32.astype(np.float32), E)
+    assert bad == 0
+    for t in range(T):
+        sm = np.exp(l32[t] - l32[t].max())
+        sm /= sm.sum()
+        assert np.allclose(w[t], sm[ids[t]], rtol=1e-12, atol=1e-15)
+        assert list(ids[t]) == sorted(range(E), key=lambda e: (-l32[t, e], e))
