@@ -93,7 +93,7 @@
 extern "C" {
 #endif
 
-#define NVFP4_MOE_ABI_VERSION 1
+#define NVFP4_MOE_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define NVFP4_MOE_API __attribute__((visibility("default")))
@@ -175,8 +175,20 @@ typedef enum {
 /* One forward call. DEVICE pointers, caller-owned.
  *   T               number of tokens, 0 <= T <= dims.max_tokens (T = 0 is a no-op)
  *   act, act_scale  activations; act_scale only for NVFP4_MOE_ACT_INT8
- *   router_logits   [T][E] f32; when NULL, topk_ids [T][K] i32 and
+ *   router_logits   [T][E] f32; when NULL, either router_w projects the layer's
+ *                   input to logits (below) or topk_ids [T][K] i32 and
  *                   topk_weights [T][K] f32 are used as given
+ *   router_w        [E][H] bf16 router projection, or NULL. With router_logits
+ *                   and topk_ids NULL, the library computes
+ *                   logits[t][e] = sum_k router_w[e][k] * x[t][k] with x the
+ *                   layer's input in FP32 -- never rounded to BF16 first: BF16
+ *                   and FP32 activations as given, int8 ones as the FP32
+ *                   product q * act_scale[t] -- and FP32 accumulation ("Strata
+ *                   NVFP4" README, "How it differs from upstream Strata": the
+ *                   router's BF16 projection takes FP32-exact inputs). Giving
+ *                   router_w together with router_logits is INVALID_ARG;
+ *                   router_w must be 16-byte aligned (else MISALIGNED).
+ *   dbg_logits      optional (may be NULL) [T][E] f32: the computed router logits
  *   out             [T][H] f32, written (OUT_F32) or accumulated into (OUT_F32_ADD)
  *   dbg_*           optional (may be NULL) copies of the routing results:
  *                   dbg_ids [T][K] i32, dbg_w [T][K] f32 (renormalised weights),
@@ -198,6 +210,8 @@ typedef struct {
     int32_t *dbg_counts;
     int32_t *dbg_offsets;
     int32_t *dbg_perm;
+    const uint16_t *router_w;   /* ABI version 2 */
+    float *dbg_logits;          /* ABI version 2 */
 } nvfp4_moe_io;
 
 /* Validates dims and weight pointers (all checks before any allocation), then

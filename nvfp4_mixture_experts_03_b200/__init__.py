@@ -54,7 +54,7 @@ class IO(C.Structure):
                 ("topk_ids", C.c_void_p), ("topk_weights", C.c_void_p),
                 ("out_type", C.c_int), ("out", C.c_void_p), ("dbg_ids", C.c_void_p),
                 ("dbg_w", C.c_void_p), ("dbg_counts", C.c_void_p), ("dbg_offsets", C.c_void_p),
-                ("dbg_perm", C.c_void_p)]
+                ("dbg_perm", C.c_void_p), ("router_w", C.c_void_p), ("dbg_logits", C.c_void_p)]
 
 
 class NVFP4MoEError(RuntimeError):
@@ -217,9 +217,11 @@ class MoELayer:
 
     def forward(self, x, *, logits=None, topk_ids=None, topk_weights=None, x_scale=None,
                 out=None, accumulate: bool = False, debug: dict | None = None,
-                workspace=None, stream=None) -> torch.Tensor:
+                workspace=None, stream=None, router_w=None) -> torch.Tensor:
         """Enqueue the layer on `stream` (default: torch's current stream).
         x: [T][H] bf16, int8 (with x_scale [T] f32) or f32 (residual stream).
+        Routing from `logits` [T][E] f32, from the router projection `router_w`
+        [E][H] bf16 of x, or from `topk_ids`/`topk_weights` as given.
         Returns `out` ([T][H] f32)."""
         T = x.shape[0]
         act_type = {torch.bfloat16: ACT_BF16, torch.int8: ACT_INT8, torch.float32: ACT_F32}[x.dtype]
@@ -229,7 +231,8 @@ class MoELayer:
         io = IO(T, act_type, _ptr(x), _ptr(x_scale), _ptr(logits), _ptr(topk_ids),
                 _ptr(topk_weights), OUT_F32_ADD if accumulate else OUT_F32, _ptr(out),
                 _ptr(dbg.get("ids")), _ptr(dbg.get("w")), _ptr(dbg.get("counts")),
-                _ptr(dbg.get("offsets")), _ptr(dbg.get("perm")))
+                _ptr(dbg.get("offsets")), _ptr(dbg.get("perm")), _ptr(router_w),
+                _ptr(dbg.get("logits")))
         ws = workspace if workspace is not None else self.workspace(T)
         rc = nvfp4_moe_forward(self.handle, io, ws.data_ptr(), ws.numel(), _stream_handle(stream))
         if rc != OK:
@@ -263,8 +266,10 @@ class MoELayer:
 
 
 def debug_buffers(T: int, E: int, K: int, device) -> dict:
-    """Optional routing outputs for checks: ids, w, counts, offsets, perm."""
+    """Optional routing outputs for checks: ids, w, counts, offsets, perm, and the
+    router projection's logits (written only when the layer computes them)."""
     i32 = dict(dtype=torch.int32, device=device)
     return {"ids": torch.empty(T, K, **i32), "w": torch.empty(T, K, dtype=torch.float32, device=device),
             "counts": torch.empty(E, **i32), "offsets": torch.empty(E + 1, **i32),
-            "perm": torch.empty(T * K, **i32)}
+            "perm": torch.empty(T * K, **i32),
+            "logits": torch.empty(T, E, dtype=torch.float32, device=device)}

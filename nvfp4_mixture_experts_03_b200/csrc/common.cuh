@@ -51,6 +51,8 @@ struct Params {
     const void *act;
     const float *act_scale;
     const float *logits;       // may be null
+    const uint16_t *router_w;  // [E][H] bf16 router projection, or null
+    float *rlogits;            // [T][E] logits the router projection writes
     const int32_t *in_ids;     // precomputed routing when logits == null
     const float *in_w;
     float *out;
@@ -414,5 +416,7 @@ cudaError_t launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &ma
 // many CTA pairs of either GEMM can be resident at once.
 cudaError_t prefill_init(int *max_clusters);
 cudaError_t decode_init();    // per device: opt the decode kernels into their shared memory
+cudaError_t router_init();    // per device: opt the router GEMM into its shared memory
+cudaError_t launch_router(const Params &p, cudaStream_t s);   // logits = x . W_r^T into p.rlogits
 
 }  // namespace nvmoe

@@ -105,7 +105,7 @@ bool use_decode(const nvfp4_moe_dims &d, int T) {
 
 struct WsLayout {
     size_t cnt, ids, wts, hist, cbase, counts, offsets, perm, inv, ptok, pw, ps, xscale, ph, phinv, tiles_gu,
-        tiles_dn, xh, h, total;
+        tiles_dn, xh, h, rlogits, total;
     int nch, max_gu, max_dn;
 };
 
@@ -143,6 +143,7 @@ WsLayout layout(const nvfp4_moe_dims &d, int T) {
     L.tiles_dn = take((size_t)L.max_dn * sizeof(Tile));
     L.xh = take(decode ? 0 : P * d.hidden * 2);   // decode stages activations in shared memory
     L.h = take(P * d.inter * 2);
+    L.rlogits = take((size_t)T * E * 4);   // router projection output (when used)
     L.total = o;
     return L;
 }
@@ -199,7 +200,8 @@ int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (major != 10) return NVFP4_MOE_ERR_NO_DEVICE;
     int pf_clusters = 0;
-    if (prefill_init(&pf_clusters) != cudaSuccess || decode_init() != cudaSuccess || !encode_fn())
+    if (prefill_init(&pf_clusters) != cudaSuccess || decode_init() != cudaSuccess ||
+        router_init() != cudaSuccess || !encode_fn())
         return NVFP4_MOE_ERR_CUDA;
     nvfp4_moe *h = new (std::nothrow) nvfp4_moe;
     if (!h) return NVFP4_MOE_ERR_CUDA;
@@ -254,11 +256,16 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     if (T == 0) return NVFP4_MOE_OK;
     if (!io->act || !io->out) return NVFP4_MOE_ERR_INVALID_ARG;
     if (io->act_type == NVFP4_MOE_ACT_INT8 && !io->act_scale) return NVFP4_MOE_ERR_INVALID_ARG;
-    if (!io->router_logits && (!io->topk_ids || !io->topk_weights)) return NVFP4_MOE_ERR_INVALID_ARG;
+    // routing source: given logits, the router projection, or given ids and weights
+    const bool router = !io->router_logits && io->router_w;
+    if (io->router_logits && io->router_w) return NVFP4_MOE_ERR_INVALID_ARG;
+    if (router && (io->topk_ids || io->topk_weights)) return NVFP4_MOE_ERR_INVALID_ARG;
+    if (!io->router_logits && !router && (!io->topk_ids || !io->topk_weights)) return NVFP4_MOE_ERR_INVALID_ARG;
     if (io->act == io->out && io->out_type != NVFP4_MOE_OUT_F32_ADD) return NVFP4_MOE_ERR_INVALID_ARG;
     if (!al16(io->act) || !al16(io->out) || (io->router_logits && !al16(io->router_logits)) ||
         (io->act_scale && !al4(io->act_scale)) || (io->topk_ids && !al4(io->topk_ids)) ||
-        (io->topk_weights && !al4(io->topk_weights)))
+        (io->topk_weights && !al4(io->topk_weights)) || (io->router_w && !al16(io->router_w)) ||
+        (io->dbg_logits && !al16(io->dbg_logits)))
         return NVFP4_MOE_ERR_MISALIGNED;
     const WsLayout L = layout(d, T);
     if (!ws || ws_bytes < L.total) return NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL;
@@ -276,6 +283,9 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     p.act = io->act;
     p.act_scale = io->act_scale;
     p.logits = io->router_logits;
+    p.router_w = io->router_w;
+    p.rlogits = io->dbg_logits ? io->dbg_logits : reinterpret_cast<float *>(b + L.rlogits);
+    if (router) p.logits = p.rlogits;
     p.in_ids = io->topk_ids;
     p.in_w = io->topk_weights;
     p.out = io->out;
@@ -341,6 +351,7 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
         // one kernel for the whole decode layer: its routing, staging and both
         // projections are not separable by events (phases 0-2 and 3-4 coincide)
         mark(0);
+        if (router && launch_router(p, s) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
         mark(1);
         mark(2);
         if (launch_decode(p, s) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
@@ -352,6 +363,7 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
         if (!make_map_f16(&map_xh, p.xh, P, d.hidden, 64) || !make_map_f16(&map_h, p.h, P, d.inter, 64))
             return NVFP4_MOE_ERR_CUDA;
         mark(0);
+        if (router && launch_router(p, s) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
         launch_route_large(p, s);
         mark(1);
         launch_prep_prefill(p, s);
@@ -448,7 +460,7 @@ int static_scratch(int dev, uint8_t **out) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p)
             return NVFP4_MOE_ERR_CUDA;
-        if (decode_init() != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
+        if (decode_init() != cudaSuccess || router_init() != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
         g_static_ptr[dev] = static_cast<uint8_t *>(p);
     }
     *out = g_static_ptr[dev];

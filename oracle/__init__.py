@@ -253,6 +253,10 @@ def forward(layer, x, *, K: int, logits=None, ids=None, wts=None, x_scale=None, 
     if router_w is not None:
         logits64 = router(router_input(x, x_scale), router_w)
         logits = logits64.astype(np.float32)
+    if _np(x).dtype == np.float32:
+        # FP32 activations (a residual stream): the experts take their nearest
+        # BF16 values, ties to even
+        x = bf16_rne_array(_np(x).astype(np.float64))
     if logits is not None:
         ids, w, bad = route(logits, K)
     else:

@@ -287,6 +287,12 @@ def make_logits(T: int, E: int, seed: int, zipf_s: float | None = None, device="
     return l.contiguous()
 
 
+def make_router_w(E: int, H: int, seed: int, std: float = 0.05, device="cpu") -> torch.Tensor:
+    """Router projection weights [E][H] bf16 ~ BF16(N(0, std^2)), one seeded stream."""
+    g = _gen(device, seed, 0x52)
+    return (torch.randn(E, H, generator=g, device=device, dtype=torch.float32) * std).to(torch.bfloat16)
+
+
 def make_topk(T: int, E: int, K: int, seed: int, device="cpu"):
     """Precomputed routing: K distinct ids per token drawn uniformly, weights a
     random positive vector normalised to 1 (FP32)."""

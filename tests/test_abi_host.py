@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings_and_version(L):
-    assert nv.nvfp4_moe_abi_version() == 1
+    assert nv.nvfp4_moe_abi_version() == 2
     for code in nv.ERR:
         assert nv.nvfp4_moe_strerror(code) not in ("", "unknown status")
     assert nv.nvfp4_moe_strerror(12345) == "unknown status"
