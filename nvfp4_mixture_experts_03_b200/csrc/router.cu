@@ -10,17 +10,19 @@
 // product of a BF16 weight and an FP32 input is exact inside the FMA; only the
 // sum rounds), lanes reduced in a fixed tree.
 //
-// Larger batches: a tcgen05 GEMM, one CTA per (128 experts, 64 tokens) tile, two
-// CTAs per SM (each hides the other's load latency).
+// Larger batches: a tcgen05 GEMM, one CTA per 64 tokens against up to 512
+// experts (four 128-row accumulators in TMEM; 256 for FP32 / int8 inputs), so a
+// token's activations are read once or twice.
 // The tensor cores take BF16 operands, so each FP32 input is split exactly into
 // three BF16 terms, x = x0 + x1 + x2 (x0 the nearest BF16 to x, x1 the nearest to
 // x - x0, x2 = x - x0 - x1, which fits in BF16), and the tile runs three MMAs per
 // K step into one FP32 accumulator: every product W * x_j is exact, the sums
 // round in FP32, as in the small-batch kernel. BF16 activations need only x0.
-// All 256 threads stage the operands (W_r rows copied, x split) into two
-// 128-byte-swizzled K-major stages of 64 K; one thread issues the MMAs and
-// commits each stage to an mbarrier that frees it; warps 0..3 read the 128 x 64
-// accumulator out of TMEM.
+// The operands reach shared memory by cp.async, in a ring of two or three
+// 128-byte-swizzled K-major stages of 64 K (BF16 activations straight into their
+// tile; FP32 / int8 ones raw, then split by all 256 threads); one thread issues
+// the MMAs and commits each stage to an mbarrier that frees it; warps 0..3 read
+// the accumulators out of TMEM.
 #include "common.cuh"
 
 namespace nvmoe {
@@ -98,11 +100,15 @@ __global__ void __launch_bounds__(kRvWarps * 32) router_gemv_kernel(Params p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * kRvWarps + warp;
     const int T = p.T, n8 = p.H / 8;
-    const int xbytes = T * p.H * act_elem_bytes(p.act_type);
-    for (int c = threadIdx.x; c < xbytes / 16; c += blockDim.x)
+    const int xbytes = T * p.H * act_elem_bytes(p.act_type), nx = xbytes / 16;
+    // every CTA copies the same rows: each starts at its own piece and wraps
+    const int x_first = (int)(((long long)blockIdx.x * 97) % nx);
+    for (int i = threadIdx.x; i < nx; i += blockDim.x) {
+        const int c = (i + x_first) % nx;
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(rv_xs + 16 * c)),
                      "l"(static_cast<const uint8_t *>(p.act) + 16 * c)
                      : "memory");
+    }
     asm volatile("cp.async.commit_group;" ::: "memory");
     float acc[kRvMaxT];
 #pragma unroll
@@ -155,17 +161,31 @@ __global__ void __launch_bounds__(kRvWarps * 32) router_gemv_kernel(Params p) {
 }
 
 // ------------------------------------------------------------------ GEMM
-constexpr int kRtM = 128;        // experts per CTA (TMEM lanes)
-constexpr int kRtN = 64;         // tokens per CTA (accumulator columns)
+// 128-expert M tiles per CTA: four (512 experts) for BF16 activations, two for
+// FP32 / int8 ones (whose stages also hold the raw rows and three part tiles),
+// so that three stages fit; more experts -> more CTAs along grid.y.
+__host__ __device__ inline int rt_mt_max(int act_type) { return act_type == NVFP4_MOE_ACT_BF16 ? 4 : 2; }
+constexpr int kRtN = 64;         // tokens per CTA (accumulator columns per M tile)
 constexpr int kRtK = 64;         // K per stage: 128 bytes of BF16 per row
 constexpr int kRtThreads = 256;
-constexpr int kRtTileA = kRtM * kRtK * 2;        // 16 KB: 128 W_r rows x 128 B
+constexpr int kRtTileA = 128 * kRtK * 2;         // 16 KB: 128 W_r rows x 128 B
 constexpr int kRtTileB = kRtN * kRtK * 2;        // 8 KB: 64 token rows x 128 B
-constexpr int kRtStage = kRtTileA + 3 * kRtTileB; // A, then the three parts of x
-constexpr int kRtSmem = 2 * kRtStage + 1024 + 64; // two stages, 1024-B alignment slack, barriers
-constexpr int kRtChunksA = kRtM * 8 / kRtThreads; // 16-byte A chunks per thread per stage (4)
-constexpr int kRtChunksB = kRtN * 8 / kRtThreads; // 8-input x chunks per thread per stage (2)
+constexpr int kRtSmemBudget = 216 * 1024;        // stages of the ring (the rest: barriers, alignment)
 constexpr uint64_t kRtWaitNs = 2000000000ull;
+
+// Bytes of one stage: A tiles, the x part tiles, and (FP32 / int8 inputs) the raw
+// activations the parts are split from.
+__host__ __device__ inline int rt_raw_bytes(int act_type) {
+    return act_type == NVFP4_MOE_ACT_BF16 ? 0 : kRtN * kRtK * (act_type == NVFP4_MOE_ACT_INT8 ? 1 : 4);
+}
+__host__ __device__ inline int rt_stage_bytes(int mt, int act_type) {
+    const int nsplit = act_type == NVFP4_MOE_ACT_BF16 ? 1 : 3;
+    return mt * kRtTileA + nsplit * kRtTileB + rt_raw_bytes(act_type);
+}
+__host__ __device__ inline int rt_stages(int mt, int act_type) {
+    const int n = kRtSmemBudget / rt_stage_bytes(mt, act_type);
+    return n < 3 ? n : 3;
+}
 
 __device__ inline void tmem_alloc1(uint32_t *slot_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -194,6 +214,12 @@ __device__ inline void tc_commit1(uint64_t *bar) {
 __host__ __device__ inline uint32_t idesc_bf16(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// 16-byte asynchronous copy; src_bytes = 0 fills the destination with zeros.
+__device__ inline void cp16(void *dst, const void *src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
 
 // x = x0 + x1 + x2 exactly, each a BF16 (bits returned).
 __device__ inline void split3(float x, uint32_t &b0, uint32_t &b1, uint32_t &b2) {
@@ -207,64 +233,75 @@ __device__ inline void split3(float x, uint32_t &b0, uint32_t &b1, uint32_t &b2)
     b2 = __bfloat16_as_ushort(h2);
 }
 
-// One thread's share of a K stage: 16-byte A chunks (8 BF16 of a W_r row) and
-// x chunks (8 inputs of a token), loaded into registers one stage ahead.
-struct RtRegs {
-    uint4 a[kRtChunksA];
-    float x[kRtChunksB][8];
-};
+// Swizzled offset (128-byte rows, 16-byte chunk c of row r at c ^ (r & 7)).
+__device__ inline int swz(int row, int ch) { return row * 128 + ((ch ^ (row & 7)) << 4); }
 
-__device__ inline void rt_load(const Params &p, int m0, int n0, int k0, RtRegs &r) {
-#pragma unroll
-    for (int i = 0; i < kRtChunksA; i++) {
-        const int c = threadIdx.x + kRtThreads * i;   // row c / 8, chunk c % 8
-        const int row = c >> 3, k = k0 + 8 * (c & 7), e = m0 + row;
-        r.a[i] = (e < p.E && k < p.H)
-                     ? __ldg(reinterpret_cast<const uint4 *>(p.router_w + (size_t)e * p.H + k))
-                     : make_uint4(0, 0, 0, 0);
+// Issues the copies of K step k0 into a stage: the CTA's W_r rows (zeros past E
+// or H) and the tokens' activations -- straight into the BF16 part tile, or raw
+// (FP32 / int8) for the split.
+__device__ inline void rt_issue(const Params &p, uint8_t *st, int mt, int m0, int n0, int k0) {
+    for (int c = threadIdx.x; c < mt * 128 * 8; c += kRtThreads) {
+        const int row = c >> 3, ch = c & 7, e = m0 + row, k = k0 + 8 * ch;
+        const bool ok = e < p.E && k < p.H;
+        cp16(st + (row >> 7) * kRtTileA + swz(row & 127, ch),
+             p.router_w + (ok ? (size_t)e * p.H + k : 0), ok ? 16 : 0);
     }
-#pragma unroll
-    for (int i = 0; i < kRtChunksB; i++) {
-        const int c = threadIdx.x + kRtThreads * i;
-        const int row = c >> 3, k = k0 + 8 * (c & 7), t = n0 + row;
-        if (t < p.T && k < p.H) {
-            router_x8(p, t, k / 8, r.x[i]);
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; j++) r.x[i][j] = 0.0f;
+    uint8_t *bt = st + mt * kRtTileA;
+    if (p.act_type == NVFP4_MOE_ACT_BF16) {
+        for (int c = threadIdx.x; c < kRtN * 8; c += kRtThreads) {
+            const int row = c >> 3, ch = c & 7, t = n0 + row, k = k0 + 8 * ch;
+            const bool ok = t < p.T && k < p.H;
+            cp16(bt + swz(row, ch), static_cast<const __nv_bfloat16 *>(p.act) + (ok ? (size_t)t * p.H + k : 0),
+                 ok ? 16 : 0);
+        }
+    } else {
+        // raw rows: kRtK elements of each token, 16-byte pieces
+        const int eb = p.act_type == NVFP4_MOE_ACT_INT8 ? 1 : 4, per = kRtK * eb / 16;
+        uint8_t *raw = bt + 3 * kRtTileB;
+        for (int c = threadIdx.x; c < kRtN * per; c += kRtThreads) {
+            const int row = c / per, piece = c - row * per, t = n0 + row;
+            const int k = k0 + piece * 16 / eb;
+            const bool ok = t < p.T && k < p.H;
+            cp16(raw + row * kRtK * eb + 16 * piece,
+                 static_cast<const uint8_t *>(p.act) + (ok ? ((size_t)t * p.H + k) * eb : 0), ok ? 16 : 0);
         }
     }
 }
 
-// Stores the registers into stage `st` in the 128-byte swizzled K-major layout
-// (16-byte chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4)).
-__device__ inline void rt_store(uint8_t *st, const RtRegs &r, int nsplit) {
-#pragma unroll
-    for (int i = 0; i < kRtChunksA; i++) {
-        const int c = threadIdx.x + kRtThreads * i;
+// FP32 / int8 stages: the raw activations -> the three exact BF16 part tiles.
+__device__ inline void rt_split(const Params &p, uint8_t *st, int mt, int n0) {
+    uint8_t *bt = st + mt * kRtTileA;
+    const uint8_t *raw = bt + 3 * kRtTileB;
+    for (int c = threadIdx.x; c < kRtN * 8; c += kRtThreads) {
         const int row = c >> 3, ch = c & 7;
-        *reinterpret_cast<uint4 *>(st + row * 128 + ((ch ^ (row & 7)) << 4)) = r.a[i];
-    }
+        float v[8];
+        if (p.act_type == NVFP4_MOE_ACT_INT8) {
+            const uint2 u = reinterpret_cast<const uint2 *>(raw + row * kRtK)[ch];
+            const uint32_t w[2] = {u.x, u.y};
+            const int t = n0 + row;
+            const float s = t < p.T ? __ldg(p.act_scale + t) : 0.0f;
 #pragma unroll
-    for (int i = 0; i < kRtChunksB; i++) {
-        const int c = threadIdx.x + kRtThreads * i;
-        const int row = c >> 3, ch = c & 7;
-        const int off = kRtTileA + row * 128 + ((ch ^ (row & 7)) << 4);
+            for (int i = 0; i < 8; i++) v[i] = __fmul_rn((float)(int8_t)(w[i >> 2] >> (8 * (i & 3))), s);
+        } else {
+            const float4 a = reinterpret_cast<const float4 *>(raw + row * kRtK * 4)[2 * ch];
+            const float4 b = reinterpret_cast<const float4 *>(raw + row * kRtK * 4)[2 * ch + 1];
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        }
         uint32_t w[3][4];
 #pragma unroll
         for (int j = 0; j < 4; j++) {
             uint32_t l0, l1, l2, h0, h1, h2;
-            split3(r.x[i][2 * j], l0, l1, l2);
-            split3(r.x[i][2 * j + 1], h0, h1, h2);
+            split3(v[2 * j], l0, l1, l2);
+            split3(v[2 * j + 1], h0, h1, h2);
             w[0][j] = l0 | (h0 << 16);
             w[1][j] = l1 | (h1 << 16);
             w[2][j] = l2 | (h2 << 16);
         }
 #pragma unroll
         for (int sp = 0; sp < 3; sp++)
-            if (sp < nsplit)
-                *reinterpret_cast<uint4 *>(st + off + sp * kRtTileB) =
-                    make_uint4(w[sp][0], w[sp][1], w[sp][2], w[sp][3]);
+            *reinterpret_cast<uint4 *>(bt + sp * kRtTileB + swz(row, ch)) =
+                make_uint4(w[sp][0], w[sp][1], w[sp][2], w[sp][3]);
     }
 }
 
@@ -280,94 +317,118 @@ __device__ inline bool rt_wait(uint64_t *bar, uint32_t parity, int32_t *status, 
     return true;
 }
 
-__global__ void __launch_bounds__(kRtThreads, 2) router_gemm_kernel(Params p) {
+// One CTA: tokens [n0, n0 + 64) against up to 4 x 128 experts from m0. A ring of
+// `ns` stages is filled by cp.async (ns - 1 K steps ahead); the stage of step
+// ks - 1 is refilled once its MMAs have completed.
+__global__ void __launch_bounds__(kRtThreads, 1) router_gemm_kernel(Params p) {
     extern __shared__ uint8_t rt_smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(rt_smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 2 * kRtStage);   // [0..1] stage free, [2] drain
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int mtx = rt_mt_max(p.act_type);
+    const int n0 = blockIdx.x * kRtN, m0 = blockIdx.y * mtx * 128;
+    const int mt = min(mtx, cdiv(p.E - m0, 128));
+    const int nsplit = p.act_type == NVFP4_MOE_ACT_BF16 ? 1 : 3;
+    const int sb = rt_stage_bytes(mt, p.act_type), ns = rt_stages(mt, p.act_type);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ns * sb);   // [0..ns) stage's MMAs done, [3] drain
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4);
     __shared__ int s_ok;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * kRtM, n0 = blockIdx.y * kRtN;
-    const int nsplit = p.act_type == NVFP4_MOE_ACT_BF16 ? 1 : 3;
     const int nk = cdiv(p.H, kRtK);
+    const uint32_t ncols = mt * kRtN <= 64 ? 64 : (mt * kRtN <= 128 ? 128 : 256);
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        mbar_init(&bars[2], 1);
+        for (int i = 0; i < 4; i++) mbar_init(&bars[i], 1);
         fence_barrier_init();
         s_ok = 1;
     }
     if (warp == 0) {
-        tmem_alloc1(tmem_slot, kRtN);
+        tmem_alloc1(tmem_slot, ncols);
         tmem_relinquish1();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t idesc = idesc_bf16(kRtM, kRtN);
+    const uint32_t idesc = idesc_bf16(128, kRtN);
 
-    // two register sets in turn: the loads of stage ks + 1 are in flight while
-    // stage ks is stored and multiplied
-    RtRegs r0, r1;
-    rt_load(p, m0, n0, 0, r0);
-    int ks = 0;
-    auto step = [&](RtRegs &cur, RtRegs &nxt) {
-        const int s = ks & 1;
-        uint8_t *st = sm + s * kRtStage;
-        if (ks + 1 < nk) rt_load(p, m0, n0, (ks + 1) * kRtK, nxt);
-        if (ks >= 2 && threadIdx.x == 0 && s_ok)   // the MMAs of step ks - 2 are done with stage s
-            s_ok = rt_wait(&bars[s], ((ks >> 1) - 1) & 1, p.status, 201);
+    // Every CTA reads the same W_r rows; each starts its sweep over K at its own
+    // step (and wraps), so that the CTAs do not all ask for the same lines at once.
+    const int k_first = (int)(((long long)blockIdx.x * 7 + blockIdx.y * 3) % nk);
+    auto kstep = [&](int j) { return (k_first + j) % nk; };
+    for (int j = 0; j < ns - 1; j++) {
+        if (j < nk) rt_issue(p, sm + j * sb, mt, m0, n0, kstep(j) * kRtK);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    for (int ks = 0; ks < nk; ks++) {
+        const int s = ks % ns;
+        uint8_t *st = sm + s * sb;
+        // this step's copies (one group committed per step; ns - 2 may stay in flight)
+        if (ns == 3) asm volatile("cp.async.wait_group 1;" ::: "memory");
+        else asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();
-        if (!s_ok) return;
-        rt_store(st, cur, nsplit);
+        if (nsplit == 3) {
+            rt_split(p, st, mt, n0);
+            __syncthreads();
+        }
         fence_proxy_async_smem();
         __syncthreads();
         if (threadIdx.x == 0) {
             tc_fence_after();
-            const uint32_t as = smem_u32(st);
+            const uint32_t as = smem_u32(st), bs = as + mt * kRtTileA;
+            for (int j = 0; j < mt; j++)
 #pragma unroll
-            for (int k16 = 0; k16 < kRtK / 16; k16++)
-                for (int sp = 0; sp < nsplit; sp++)
-                    tc_mma_bf16(tmem, smem_desc_sw128(as + 32 * k16),
-                                smem_desc_sw128(as + kRtTileA + sp * kRtTileB + 32 * k16), idesc,
-                                (ks | k16 | sp) != 0);
+                for (int k16 = 0; k16 < kRtK / 16; k16++)
+                    for (int sp = 0; sp < nsplit; sp++)
+                        tc_mma_bf16(tmem + j * kRtN, smem_desc_sw128(as + j * kRtTileA + 32 * k16),
+                                    smem_desc_sw128(bs + sp * kRtTileB + 32 * k16), idesc,
+                                    (ks | k16 | sp) != 0);
             tc_commit1(&bars[s]);
+            // the stage of step ks - 1 is refilled (for step ks + ns - 1) once its MMAs are done
+            if (ks >= 1 && s_ok) {
+                const int ps = (ks - 1) % ns, use = (ks - 1) / ns;
+                s_ok = rt_wait(&bars[ps], use & 1, p.status, 201);
+            }
         }
-        ks++;
-    };
-    while (ks < nk && s_ok) {
-        step(r0, r1);
-        if (ks >= nk || !s_ok) break;
-        step(r1, r0);
+        __syncthreads();
+        if (!s_ok) break;
+        const int kn = ks + ns - 1;
+        if (kn < nk) rt_issue(p, sm + (kn % ns) * sb, mt, m0, n0, kstep(kn) * kRtK);
+        asm volatile("cp.async.commit_group;" ::: "memory");
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     // every MMA issued so far has completed once the drain barrier fires
     if (threadIdx.x == 0) {
-        tc_commit1(&bars[2]);
-        if (!rt_wait(&bars[2], 0, p.status, 202)) s_ok = 0;
+        tc_commit1(&bars[3]);
+        if (!rt_wait(&bars[3], 0, p.status, 202)) s_ok = 0;
     }
     __syncthreads();
     tc_fence_after();
     if (warp < 4 && s_ok) {
-        const int e = m0 + 32 * warp + lane;
+        for (int j = 0; j < mt; j++) {
+            const int e = m0 + 128 * j + 32 * warp + lane;
 #pragma unroll 1
-        for (int c0 = 0; c0 < kRtN; c0 += 32) {
-            uint32_t v[32];
-            tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + c0, v);
-            tmem_ld_wait();
-            if (e < p.E) {
+            for (int c0 = 0; c0 < kRtN; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + j * kRtN + c0, v);
+                tmem_ld_wait();
+                if (e < p.E) {
 #pragma unroll
-                for (int j = 0; j < 32; j++) {
-                    const int t = n0 + c0 + j;
-                    if (t < p.T) p.rlogits[(size_t)t * p.E + e] = __uint_as_float(v[j]);
+                    for (int q = 0; q < 32; q++) {
+                        const int t = n0 + c0 + q;
+                        if (t < p.T) p.rlogits[(size_t)t * p.E + e] = __uint_as_float(v[q]);
+                    }
                 }
             }
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc1(tmem, kRtN);
+    if (warp == 0) tmem_dealloc1(tmem, ncols);
+}
+
+static size_t rt_smem_for(int E, int act_type) {
+    const int mtx = rt_mt_max(act_type);
+    const int mt = E < mtx * 128 ? cdiv(E, 128) : mtx;
+    return (size_t)rt_stages(mt, act_type) * rt_stage_bytes(mt, act_type) + 1024 + 64;
 }
 
 cudaError_t launch_router(const Params &p, cudaStream_t s) {
@@ -376,14 +437,15 @@ cudaError_t launch_router(const Params &p, cudaStream_t s) {
         router_gemv_kernel<<<cdiv(p.E, kRvWarps), kRvWarps * 32, xbytes, s>>>(p);
         return cudaGetLastError();
     }
-    const dim3 grid(cdiv(p.E, kRtM), cdiv(p.T, kRtN));
-    router_gemm_kernel<<<grid, kRtThreads, kRtSmem, s>>>(p);
+    const dim3 grid(cdiv(p.T, kRtN), cdiv(p.E, rt_mt_max(p.act_type) * 128));
+    router_gemm_kernel<<<grid, kRtThreads, rt_smem_for(p.E, p.act_type), s>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t router_init() {
     const cudaError_t a =
-        cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRtSmem);
+        cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kRtSmemBudget + 1024 + 64);
     const cudaError_t b =
         cudaFuncSetAttribute(router_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRvSmemMax);
     return a != cudaSuccess ? a : b;
