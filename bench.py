@@ -653,21 +653,27 @@ def run_reference(args, ws, rank):
 def ncu_target(case):
     """A few forwards of one case on cuda:0, for an ncu capture (-k selects the
     kernel, -s skips the first launches). prefill8k: 3 forwards of the 8192-token
-    chunk; decode8: 6 forwards of 8 tokens on the decode layer."""
+    chunk; decode8: 6 forwards of 8 tokens on the decode layer; router8k /
+    router8: 3 forwards of 8192 / 8 tokens whose logits come from the layer's
+    router projection (BF16 W_r [512][2048])."""
     import nvfp4_mixture_experts_03_b200 as nv
     dev = torch.device("cuda", 0)
-    wl = synth.CONFIGS["prefill8k" if case == "prefill8k" else "decode"]
+    wl = synth.CONFIGS["prefill8k" if case in ("prefill8k", "router8k") else "decode"]
     d = wl.dims
     seed = synth.workload_seed(wl)
     layer = synth.make_layer(d, seed, device=dev)
-    T = wl.tokens[0] if case == "prefill8k" else 8
+    T = wl.tokens[0] if case in ("prefill8k", "router8k") else 8
     x = synth.make_x_bf16(T, d.H, seed, outliers=wl.outliers, device=dev)
     logits = synth.make_logits(T, d.E, seed, zipf_s=wl.zipf_s, device=dev)
+    wr = synth.make_router_w(d.E, d.H, seed, device=dev) if case.startswith("router") else None
     m = nv.MoELayer.from_layer(layer, top_k=d.K, max_tokens=T)
     out = torch.empty(T, d.H, device=dev)
     ws = m.workspace(T)
-    for _ in range(3 if case == "prefill8k" else 6):
-        m.forward(x, logits=logits, out=out, workspace=ws)
+    for _ in range(6 if case == "decode8" else 3):
+        if wr is None:
+            m.forward(x, logits=logits, out=out, workspace=ws)
+        else:
+            m.forward(x, router_w=wr, out=out, workspace=ws)
     torch.cuda.synchronize()
     st = m.status()
     m.close()
@@ -692,7 +698,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-subrecords", action="store_true",
                     help="skip the 32K W4A8 and 48-layer stack sub-records of the default run")
-    ap.add_argument("--ncu-target", choices=["prefill8k", "decode8"],
+    ap.add_argument("--ncu-target", choices=["prefill8k", "decode8", "router8k", "router8"],
                     help="profiling aid: a few untimed forwards of one case (for ncu), no JSON")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
