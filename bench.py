@@ -594,6 +594,26 @@ def run_stack(args, ws, rank, local):
                         "unique_experts": uniq, "GBps": round(gbs, 1), "frac": round(gbs / pk["hbm_gbs"], 4),
                         "timed_launches": reps * wl.layers}
         del g
+        xg = xd.clone()   # the per-layer graph's result
+        # the same 48 layers as ONE kernel launch (nvfp4_moe_forward_decode_stack)
+        lga = torch.stack(lgd).contiguous()
+        for _ in range(3):
+            xd.copy_(xd0)
+            nv.decode_stack(models, xd, lga, workspace=wsb)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(reps):
+            xd.copy_(xd0)
+            nv.decode_stack(models, xd, lga, workspace=wsb)
+        b.record()
+        torch.cuda.synchronize()
+        assert models[0].status() == 0
+        pms = a.elapsed_time(b) / reps
+        pgbs = uniq * per_expert / (pms / 1e3) / 1e9
+        dec[f"T{T}"]["one_launch"] = {"tokens_per_s": round(T / (pms / 1e3), 1),
+                                      "ms_per_token_step": round(pms, 3), "GBps": round(pgbs, 1),
+                                      "frac": round(pgbs / pk["hbm_gbs"], 4), "timed_launches": reps,
+                                      "same_bits_as_per_layer": bool(torch.equal(xg, xd))}
     dec["peak"] = {"hbm_gbs": pk["hbm_gbs"], "source": pk_src}
     res["decode_stack"] = dec
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -601,7 +621,8 @@ def run_stack(args, ws, rank, local):
         res["cpu_baseline"] = oracle_baseline(layers[0].to("cpu"), x0.to(torch.bfloat16).cpu(),
                                               lgp[0].cpu(), d.K, Tp, args.cpu_seconds,
                                               layers=wl.layers)
-    n_dec = sum(v["timed_launches"] for k, v in dec.items() if k.startswith("T"))
+    n_dec = sum(v["timed_launches"] + v["one_launch"]["timed_launches"]
+                for k, v in dec.items() if k.startswith("T"))
     res["gpu_launches"] += n_dec
     res["gpu_launches_by_region"]["decode_timed"] = n_dec
     for mm in models:

@@ -94,6 +94,7 @@ extern "C" {
 #endif
 
 #define NVFP4_MOE_ABI_VERSION 2
+#define NVFP4_MOE_MAX_STACK 64   /* layers of one nvfp4_moe_forward_decode_stack call */
 
 #if defined(__GNUC__)
 #define NVFP4_MOE_API __attribute__((visibility("default")))
@@ -295,6 +296,28 @@ NVFP4_MOE_API int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events
 NVFP4_MOE_API int nvfp4_moe_forward_decode_static(const nvfp4_moe_dims *dims,
                                                   const nvfp4_moe_weights *weights,
                                                   const nvfp4_moe_io *io, void *stream);
+
+/* Decode through a stack of layers in ONE kernel launch (T <= 8), over the FP32
+ * residual stream: x <- x + layer_l(bf16(x)) for l = 0..n_layers-1, in place.
+ * The pages measure the cost of launch gaps ("Strata NVFP4" README, "How it
+ * differs from upstream Strata", the prompt-reading bullet: about 10 us idle
+ * per wait); here the layers follow each other inside one kernel, separated by
+ * grid barriers, with no launch between them.
+ *   layers      n_layers handles (1 <= n_layers <= NVFP4_MOE_MAX_STACK) of
+ *               identical dims on one device, each with max_tokens >= T; each
+ *               layer's weights come from its handle; the status block and
+ *               decode counters of layers[0] are used (read its get_status).
+ *   io          act_type NVFP4_MOE_ACT_F32, out_type NVFP4_MOE_OUT_F32_ADD,
+ *               act == out ([T][H] f32, updated in place); router_logits
+ *               [n_layers][T][E] f32, layer l's at offset l*T*E; no router_w,
+ *               no topk ids/weights, no dbg_* outputs (else INVALID_ARG).
+ *   workspace   as for nvfp4_moe_forward on layers[0] with this T.
+ * Returns UNSUPPORTED_DIMS when the layer does not take the decode kernel.
+ * Every layer's arithmetic is that of nvfp4_moe_forward: the result equals
+ * n_layers forward calls bit for bit. */
+NVFP4_MOE_API int nvfp4_moe_forward_decode_stack(nvfp4_moe_t *const *layers, int32_t n_layers,
+                                                 const nvfp4_moe_io *io, void *workspace,
+                                                 size_t ws_bytes, void *stream);
 
 /* Frees the handle, its status block and decode state. Never touches the
  * borrowed weights. */

@@ -31,7 +31,7 @@ MAX_TOPK = 16
 EXPORTS = ("nvfp4_moe_create", "nvfp4_moe_workspace_bytes", "nvfp4_moe_forward",
            "nvfp4_moe_get_status", "nvfp4_moe_destroy", "nvfp4_moe_strerror",
            "nvfp4_moe_abi_version", "nvfp4_moe_set_phase_events",
-           "nvfp4_moe_forward_decode_static",
+           "nvfp4_moe_forward_decode_static", "nvfp4_moe_forward_decode_stack",
            "nvfp4_moe_test_set_flags", "nvfp4_moe_test_fail_alloc", "nvfp4_moe_test_last_detail")
 TEST_DECODE_STALL = 1   # include/nvfp4_moe_test.h
 PHASE_EVENTS = 5
@@ -92,6 +92,9 @@ def lib() -> C.CDLL:
         L.nvfp4_moe_set_phase_events.argtypes = [C.c_void_p, C.POINTER(C.c_void_p), C.c_int32]
         L.nvfp4_moe_test_last_detail.restype = C.c_int
         L.nvfp4_moe_test_last_detail.argtypes = [C.c_void_p]
+        L.nvfp4_moe_forward_decode_stack.restype = C.c_int
+        L.nvfp4_moe_forward_decode_stack.argtypes = [C.POINTER(C.c_void_p), C.c_int32, C.POINTER(IO),
+                                                     C.c_void_p, C.c_size_t, C.c_void_p]
         L.nvfp4_moe_forward_decode_static.restype = C.c_int
         L.nvfp4_moe_forward_decode_static.argtypes = [C.POINTER(Dims), C.POINTER(Weights),
                                                       C.POINTER(IO), C.c_void_p]
@@ -157,6 +160,28 @@ def nvfp4_moe_test_last_detail(handle: int) -> int:
 def nvfp4_moe_test_fail_alloc(n: int) -> None:
     """Test hook: the n-th device allocation of later creates fails (then disarms)."""
     lib().nvfp4_moe_test_fail_alloc(C.c_int32(n))
+
+
+def nvfp4_moe_forward_decode_stack(handles, io: IO, workspace: int, ws_bytes: int, stream: int) -> int:
+    """One launch for a stack of decode layers over the FP32 residual stream."""
+    arr = (C.c_void_p * len(handles))(*handles)
+    return lib().nvfp4_moe_forward_decode_stack(arr, len(handles), C.byref(io), C.c_void_p(workspace),
+                                                C.c_size_t(ws_bytes), C.c_void_p(stream))
+
+
+def decode_stack(layers, x, logits, *, workspace=None, stream=None):
+    """x <- x + layer_l(bf16(x)) for every MoELayer in `layers`, in place, in one
+    kernel launch. x: [T][H] f32 (T <= 8); logits: [L][T][E] f32. Returns x."""
+    T = x.shape[0]
+    ws = workspace if workspace is not None else layers[0].workspace(T)
+    act_type = {torch.bfloat16: ACT_BF16, torch.int8: ACT_INT8, torch.float32: ACT_F32}[x.dtype]
+    io = IO(T, act_type, _ptr(x), None, _ptr(logits), None, None, OUT_F32_ADD, _ptr(x),
+            None, None, None, None, None, None, None)
+    rc = nvfp4_moe_forward_decode_stack([m.handle for m in layers], io, ws.data_ptr(), ws.numel(),
+                                        _stream_handle(stream))
+    if rc != OK:
+        raise NVFP4MoEError(rc, "nvfp4_moe_forward_decode_stack")
+    return x
 
 
 def nvfp4_moe_forward_decode_static(dims: Dims, weights: Weights, io: IO, stream: int) -> int:

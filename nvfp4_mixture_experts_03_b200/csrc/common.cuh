@@ -396,6 +396,16 @@ void launch_route_large(const Params &p, cudaStream_t s);
 void launch_prep_prefill(const Params &p, cudaStream_t s);
 void launch_combine(const Params &p, cudaStream_t s);   // prefill: per-token sum of the K pair rows
 cudaError_t launch_decode(const Params &p, cudaStream_t s);   // the whole T <= 8 layer
+// One layer's weight planes, for a decode stack.
+struct DecLayerPtrs {
+    const uint8_t *gate_codes, *up_codes, *gate_scales, *up_scales;
+    const float *gate_global, *up_global;
+    const uint8_t *down_codes, *down_scales;
+    const float *down_global;
+};
+// n decode layers in one launch over the FP32 residual stream
+cudaError_t launch_decode_stack(const Params &p, const DecLayerPtrs *layers, int n, const float *logits,
+                                cudaStream_t s);
 int decode_grid();                                 // CTAs of the decode kernel (one per SM)
 constexpr int kDecWarpsPerCta = 16;                // warps of a decode CTA
 // Whether the decode kernel's shared-memory plan holds layers of these dims (else

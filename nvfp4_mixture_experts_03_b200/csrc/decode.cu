@@ -88,6 +88,16 @@ constexpr int kSlots = NVFP4_MOE_DECODE_MAX_T;
 
 constexpr uint64_t kDecWaitNs = 200000000ull;   // grid barrier wait limit (200 ms)
 
+// The weight planes and router logits of the layer being run (in shared memory:
+// a stack of layers swaps them per layer, the parameters stay constant).
+struct DecLayer {
+    const uint8_t *gate_codes, *up_codes, *gate_scales, *up_scales;
+    const float *gate_global, *up_global;
+    const uint8_t *down_codes, *down_scales;
+    const float *down_global;
+    const float *logits;
+};
+
 // Per-CTA routing state of the decode kernel.
 struct DecRoute {
     int ids[kMaxPairs];
@@ -115,7 +125,8 @@ struct DecRoute {
 // plus the number of earlier tokens in the mask. `ex` and `sc` are E ints of
 // shared scratch each. Warps kSlots.. (which route no token) run `side` meanwhile.
 template <int NPER, class Side>
-__device__ void cta_route(const Params &p, DecRoute &R, bool report, int *ex, int *sc, Side side) {
+__device__ void cta_route(const Params &p, const float *logits, DecRoute &R, bool report, int *ex, int *sc,
+                          Side side) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = p.T * p.K, E = p.E;
     for (int i = threadIdx.x; i < kMaxPairs * kSlots; i += blockDim.x) R.upos[i] = -1;
@@ -125,9 +136,9 @@ __device__ void cta_route(const Params &p, DecRoute &R, bool report, int *ex, in
     if (warp < p.T) {
         int id;
         float w;
-        if (p.logits) {
+        if (logits) {
             bool finite;
-            warp_topk<NPER>(p.logits + (size_t)warp * E, E, p.K, lane, id, w, finite);
+            warp_topk<NPER>(logits + (size_t)warp * E, E, p.K, lane, id, w, finite);
             if (!finite && report && lane == 0) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, warp);
         } else {
             const bool ok = warp_given(p.in_ids + (size_t)warp * p.K, p.in_w + (size_t)warp * p.K,
@@ -217,6 +228,13 @@ struct DecPlan {
     int last;   // this CTA finished last (resets the counters)
 };
 
+constexpr int kMaxStackLayers = NVFP4_MOE_MAX_STACK;
+struct DecStack {
+    int32_t n;
+    const float *logits;   // [n][T][E]
+    DecLayer layer[kMaxStackLayers];
+};
+
 // Gate/up weights of one warp's chunk: rows g (gate) and g+8 (up), up to
 // kGuRounds rounds.
 struct GuBuf {
@@ -243,14 +261,14 @@ __device__ inline Chunk take_chunk(int &x, int end, int R) {
 
 // Weight loads of rounds [c.r0, c.r1) of granule P.gb + c.item; 16-byte pieces
 // past the row's end (H not a multiple of 128) are zero, with zero scales.
-__device__ inline void gu_issue(const Params &p, const DecRoute &R, const DecPlan &P, const Chunk &c,
-                                int g, int q, GuBuf &b) {
+__device__ inline void gu_issue(const Params &p, const DecLayer &W, const DecRoute &R, const DecPlan &P,
+                                const Chunk &c, int g, int q, GuBuf &b) {
     if (c.r1 == 0) return;
     const int per_u = p.I / 8, gi = P.gb + c.item, u = gi / per_u;
     const size_t ra = (size_t)R.uniq[u] * p.I + (gi - u * per_u) * 8 + g;
     const int kb = p.H / 2;
-    const uint8_t *ca_p = p.gate_codes + ra * kb, *cb_p = p.up_codes + ra * kb;
-    const uint8_t *sa_p = p.gate_scales + ra * (p.H / 16), *sb_p = p.up_scales + ra * (p.H / 16);
+    const uint8_t *ca_p = W.gate_codes + ra * kb, *cb_p = W.up_codes + ra * kb;
+    const uint8_t *sa_p = W.gate_scales + ra * (p.H / 16), *sb_p = W.up_scales + ra * (p.H / 16);
 #pragma unroll
     for (int j = 0; j < kGuRounds; j++) {
         const int r = c.r0 + j;
@@ -323,16 +341,16 @@ __device__ inline void dn_next(DnCur &c, int U, int R2) {
 
 // Loads of the n <= kDnUnits down units from c on; 16-byte pieces past the row's
 // end (I not a multiple of 128) are zero, with zero scales.
-__device__ inline void dn_issue(const Params &p, const DecRoute &R, int rb0, DnCur c, int n, int g, int q,
-                                DnBuf &b) {
+__device__ inline void dn_issue(const Params &p, const DecLayer &W, const DecRoute &R, int rb0, DnCur c,
+                                int n, int g, int q, DnBuf &b) {
     const int H = p.H, I = p.I, R2 = cdiv(I, 128), U = R.U;
 #pragma unroll
     for (int j = 0; j < kDnUnits; j++) {
         if (j < n) {
             if (64 * c.r + 16 * q < I / 2) {
                 const size_t ra = (size_t)R.uniq[c.u] * H + 16 * (rb0 + c.rbl) + g;
-                const uint8_t *cp = p.down_codes + ra * (I / 2) + 64 * c.r + 16 * q;
-                const uint8_t *sp = p.down_scales + ra * (I / 16) + 8 * c.r + 2 * q;
+                const uint8_t *cp = W.down_codes + ra * (I / 2) + 64 * c.r + 16 * q;
+                const uint8_t *sp = W.down_scales + ra * (I / 16) + 8 * c.r + 2 * q;
                 b.ca[j] = ldg_stream(cp);
                 b.cb[j] = ldg_stream(cp + 8 * (I / 2));
                 b.s[j] = (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sp)) |
@@ -418,11 +436,34 @@ __device__ inline int owner(int n, int W, int x) {
     return w;
 }
 
+// Generation-counting grid barrier: thread 0 of every CTA arrives; the last to
+// arrive resets the count and bumps the generation word the others wait on
+// (bounded). `gen` (thread 0's copy) is the generation being waited out; it
+// advances with each barrier. Returns, in every thread, whether it completed.
+__device__ inline bool grid_barrier(const Params &p, int32_t *ds, int &gen, int where, bool arrive,
+                                    int *ok_smem) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        bool open = false;
+        if (arrive && atomicAdd(ds + kDsArrive, 1) == (int)gridDim.x - 1) {
+            atomicExch(ds + kDsArrive, 0);
+            __threadfence();
+            atomicAdd(ds + kDsGen, 1);
+            open = true;
+        }
+        *ok_smem = open || wait_ne(ds + kDsGen, gen, p.status, where);
+        gen++;
+        __threadfence();
+    }
+    __syncthreads();
+    return *ok_smem != 0;
+}
+
+// One decode layer (routing, gate/up + SwiGLU, grid barrier, down + combine).
 template <int NPER>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) {
-    extern __shared__ __align__(16) uint8_t dsm[];
-    __shared__ DecRoute R;
-    __shared__ DecPlan P;
+__device__ __forceinline__ void decode_body(const Params &p, const DecLayer &W, DecRoute &R, DecPlan &P,
+                                            uint8_t *dsm, int &gen) {
     const int H = p.H, I = p.I, T = p.T;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int ld1 = dec_ld1(H), ld2 = dec_ld2(I);
@@ -437,12 +478,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     float *gsc = reinterpret_cast<float *>(scratch + 2 * p.E);    // [gate, up, down][E] global scales
     int32_t *ds = p.dstate;
 
-    // Everything this layer reads may come from the previous kernel in the stream.
-    grid_dep_wait();
-    // this launch's barrier generation: no CTA can open the next one before every
-    // CTA (this one included) has arrived, hence read it
-    const int gen0 = threadIdx.x == 0 ? *reinterpret_cast<volatile int32_t *>(ds + kDsGen) : 0;
-
     // While warps 0..T-1 route, warps 8..15 stage the activations: per-token amax
     // -> power-of-two shift -> F16 in shared memory (columns past H and the zero
     // row T are zero), and fetch every expert's three global scales.
@@ -450,9 +485,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     auto stage = [&]() {
         const int st = threadIdx.x - kSlots * 32, sw = st >> 5, nst = kDecThreads - kSlots * 32;
         for (int e = st; e < p.E; e += nst) {
-            gsc[e] = p.gate_global[e];
-            gsc[p.E + e] = p.up_global[e];
-            gsc[2 * p.E + e] = p.down_global[e];
+            gsc[e] = W.gate_global[e];
+            gsc[p.E + e] = W.up_global[e];
+            gsc[2 * p.E + e] = W.down_global[e];
         }
         const int h8 = H / 8, p8 = ld1 / 8;
         for (int c = st; c < T * (p8 - h8) + p8; c += nst) {
@@ -494,7 +529,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
             R.hexp[st] = h_exp_for(am);
         }
     };
-    cta_route<NPER>(p, R, blockIdx.x == 0, scratch, scratch + p.E, stage);
+    cta_route<NPER>(p, W.logits, R, blockIdx.x == 0, scratch, scratch + p.E, stage);
     const int U = R.U;
     const int n8 = U * (I / 8);
     const int gb = (int)((long long)n8 * blockIdx.x / gridDim.x);
@@ -515,7 +550,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     GuBuf buf0, buf1;
     {
         const DecPlan Pl{gb, ge, 0, 0};
-        gu_issue(p, R, Pl, cur, g, q, buf0);
+        gu_issue(p, W, R, Pl, cur, g, q, buf0);
     }
 
     __syncthreads();   // P is read by every warp from here on
@@ -531,7 +566,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
         const __half *xrow = xs + (size_t)(g < T ? g : T) * ld1 + 32 * q;
         auto step = [&](GuBuf &b, GuBuf &nb) {
             const Chunk nxt = take_chunk(x1, b1, R1);
-            gu_issue(p, R, P, nxt, g, q, nb);
+            gu_issue(p, W, R, P, nxt, g, q, nb);
 #pragma unroll
             for (int j = 0; j < kGuRounds; j++) {
                 const int r = cur.r0 + j;
@@ -572,7 +607,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     int a2, b2;
     share(n2, warp, kDecWarps, a2, b2);
     DnBuf d0, d1;
-    dn_issue(p, R, rb0, dn_cur(a2, U, R2), min(kDnUnits, b2 - a2), g, q, d0);
+    dn_issue(p, W, R, rb0, dn_cur(a2, U, R2), min(kDnUnits, b2 - a2), g, q, d0);
     __syncthreads();
     // granules split between warps: their parts summed in warp order
     for (int j = warp; j < ge - gb; j += kDecWarps) {
@@ -602,22 +637,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
 
     // grid barrier: every CTA's h is stored (and every CTA has read the
     // activations: out may alias them)
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        // the last CTA to arrive resets the count and opens the next generation
-        bool open = false;
-        if (!((p.test_flags & NVFP4_MOE_TEST_DECODE_STALL) && blockIdx.x == 0) &&
-            atomicAdd(ds + kDsArrive, 1) == (int)gridDim.x - 1) {
-            atomicExch(ds + kDsArrive, 0);
-            __threadfence();
-            atomicAdd(ds + kDsGen, 1);
-            open = true;
-        }
-        P.ok = open || wait_ne(ds + kDsGen, gen0, p.status, 101);
-        __threadfence();
-    }
-    __syncthreads();
+    grid_barrier(p, ds, gen, 101, !((p.test_flags & NVFP4_MOE_TEST_DECODE_STALL) && blockIdx.x == 0),
+                 &P.ok);
     if (P.ok && n2 > 0) {
         // every pair's h row, K past I zero, then a zero row for absent tokens
         const int per_row = ld2 / 8, P2 = T * p.K;   // 16-byte pieces per row; pairs
@@ -647,7 +668,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
                 DnCur ic = cc;   // the next chunk starts kDnUnits units on
 #pragma unroll
                 for (int j = 0; j < kDnUnits; j++) dn_next(ic, U, R2);
-                dn_issue(p, R, rb0, ic, min(kDnUnits, b2 - xn), g, q, nb);
+                dn_issue(p, W, R, rb0, ic, min(kDnUnits, b2 - xn), g, q, nb);
             }
 #pragma unroll
             for (int j = 0; j < kDnUnits; j++) {
@@ -718,7 +739,57 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) 
     warp_report(p, bad2, kNfOut);
 
     if (blockIdx.x == 0) publish_route(p, R);
+}
+
+template <int NPER>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_layer_kernel(Params p) {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ DecRoute R;
+    __shared__ DecPlan P;
+    // Everything this layer reads may come from the previous kernel in the stream.
+    grid_dep_wait();
+    // this launch's barrier generation: no CTA can open the next one before every
+    // CTA (this one included) has arrived, hence read it
+    int gen = threadIdx.x == 0 ? *reinterpret_cast<volatile int32_t *>(p.dstate + kDsGen) : 0;
+    __shared__ DecLayer W;
+    if (threadIdx.x == 0)
+        W = DecLayer{p.gate_codes, p.up_codes, p.gate_scales, p.up_scales, p.gate_global,
+                     p.up_global, p.down_codes, p.down_scales, p.down_global, p.logits};
+    __syncthreads();
+    decode_body<NPER>(p, W, R, P, dsm, gen);
     // The next layer's grid may launch once every CTA is here.
+    grid_dep_launch();
+}
+
+// A stack of decode layers in one launch over the FP32 residual stream
+// (x <- x + layer_l(bf16(x)), in place): per layer its weights and router logits
+// from the table, then a second grid barrier so that every row of x is final
+// before the next layer reads it.
+template <int NPER>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_stack_kernel(const Params p, const DecStack st) {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ DecRoute R;
+    __shared__ DecPlan P;
+    grid_dep_wait();
+    int gen = threadIdx.x == 0 ? *reinterpret_cast<volatile int32_t *>(p.dstate + kDsGen) : 0;
+    __shared__ DecLayer W;
+    // The parameters are read from shared memory inside the loop: values the
+    // compiler would otherwise hoist out of it stay in registers across every
+    // layer and spill.
+    __shared__ Params Ps;
+    if (threadIdx.x == 0) Ps = p;
+#pragma unroll 1
+    for (int l = 0; l < st.n; l++) {
+        __syncthreads();   // every thread is done with the previous layer's W
+        if (threadIdx.x == 0) {
+            W = st.layer[l];
+            W.logits = st.logits + (size_t)l * p.T * p.E;
+        }
+        __syncthreads();
+        decode_body<NPER>(Ps, W, R, P, dsm, gen);
+        if (!P.ok) break;   // a wait gave up (TIMEOUT latched): the rest is not run
+        if (l + 1 < st.n && !grid_barrier(Ps, Ps.dstate, gen, 102, true, &P.ok)) break;
+    }
     grid_dep_launch();
 }
 
@@ -770,6 +841,43 @@ static cudaError_t launch_layer(const Params &p, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, decode_layer_kernel<NPER>, p);
 }
 
+template <int NPER>
+static cudaError_t launch_stack(const Params &p, const DecStack &st, cudaStream_t s) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(decode_grid());
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = decode_smem_for(p.T, p.K, p.E, p.H, p.I);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_stack_kernel<NPER>, p, st);
+}
+
+// p: the stack's common parameters (the first layer's weights, which the
+// kernel replaces per layer); layers / logits: the table.
+cudaError_t launch_decode_stack(const Params &p, const DecLayerPtrs *layers, int n, const float *logits,
+                                cudaStream_t s) {
+    if (n < 1 || n > kMaxStackLayers) return cudaErrorInvalidValue;
+    DecStack st{};
+    st.n = n;
+    st.logits = logits;
+    for (int l = 0; l < n; l++) {
+        const DecLayerPtrs &w = layers[l];
+        st.layer[l] = DecLayer{w.gate_codes, w.up_codes, w.gate_scales, w.up_scales, w.gate_global,
+                               w.up_global, w.down_codes, w.down_scales, w.down_global, nullptr};
+    }
+    const int nper = cdiv(p.E, 32);
+    if (nper <= 1) return launch_stack<1>(p, st, s);
+    if (nper <= 2) return launch_stack<2>(p, st, s);
+    if (nper <= 4) return launch_stack<4>(p, st, s);
+    if (nper <= 8) return launch_stack<8>(p, st, s);
+    if (nper <= 16) return launch_stack<16>(p, st, s);
+    return launch_stack<32>(p, st, s);
+}
+
 cudaError_t launch_decode(const Params &p, cudaStream_t s) {
     const int n = cdiv(p.E, 32);
     if (n <= 1) return launch_layer<1>(p, s);
@@ -784,6 +892,12 @@ cudaError_t decode_init() {
     // dynamic shared memory above the 48 KB default (the activations grow with H)
     const int big = (int)kDecSmemMax;
     const cudaError_t r[] = {
+        cudaFuncSetAttribute(decode_stack_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
+        cudaFuncSetAttribute(decode_stack_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
+        cudaFuncSetAttribute(decode_stack_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
+        cudaFuncSetAttribute(decode_stack_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
+        cudaFuncSetAttribute(decode_stack_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
+        cudaFuncSetAttribute(decode_stack_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
         cudaFuncSetAttribute(decode_layer_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
         cudaFuncSetAttribute(decode_layer_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),
         cudaFuncSetAttribute(decode_layer_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, big),

@@ -242,8 +242,11 @@ size_t nvfp4_moe_workspace_bytes(const nvfp4_moe_t *h, int32_t T) {
     return layout(h->d, T).total;
 }
 
-int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t ws_bytes,
-                      void *stream) {
+// Checks a forward call and fills its kernel parameters (everything but the
+// launches). Returns NVFP4_MOE_OK, kNothingToDo for T = 0, or an error.
+constexpr int kNothingToDo = 1;
+static int prepare_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t ws_bytes, Params &p,
+                           bool &decode, bool &router) {
     if (!h || !io) return NVFP4_MOE_ERR_INVALID_ARG;
     const nvfp4_moe_dims &d = h->d;
     const int T = io->T;
@@ -253,11 +256,11 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
         return NVFP4_MOE_ERR_INVALID_ARG;
     if (io->out_type != NVFP4_MOE_OUT_F32 && io->out_type != NVFP4_MOE_OUT_F32_ADD)
         return NVFP4_MOE_ERR_INVALID_ARG;
-    if (T == 0) return NVFP4_MOE_OK;
+    if (T == 0) return kNothingToDo;
     if (!io->act || !io->out) return NVFP4_MOE_ERR_INVALID_ARG;
     if (io->act_type == NVFP4_MOE_ACT_INT8 && !io->act_scale) return NVFP4_MOE_ERR_INVALID_ARG;
     // routing source: given logits, the router projection, or given ids and weights
-    const bool router = !io->router_logits && io->router_w;
+    router = !io->router_logits && io->router_w;
     if (io->router_logits && io->router_w) return NVFP4_MOE_ERR_INVALID_ARG;
     if (router && (io->topk_ids || io->topk_weights)) return NVFP4_MOE_ERR_INVALID_ARG;
     if (!io->router_logits && !router && (!io->topk_ids || !io->topk_weights)) return NVFP4_MOE_ERR_INVALID_ARG;
@@ -272,7 +275,7 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     if (reinterpret_cast<uintptr_t>(ws) & 255) return NVFP4_MOE_ERR_MISALIGNED;
 
     uint8_t *b = static_cast<uint8_t *>(ws);
-    Params p{};
+    p = Params{};
     p.T = T;
     p.E = d.n_experts;
     p.H = d.hidden;
@@ -327,13 +330,25 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
     p.max_tiles_gu = L.max_gu;
     p.max_tiles_dn = L.max_dn;
     p.test_flags = h->test_flags;
-    const bool decode = use_decode(d, T);
+    decode = use_decode(d, T);
     if (decode) {
         if (!h->dstate) return NVFP4_MOE_ERR_INVALID_ARG;
         p.dstate = reinterpret_cast<int32_t *>(h->dstate);
         p.dec_union = (int32_t)decode_union_bytes(T, d.top_k, d.hidden, d.inter);
     }
 
+    return NVFP4_MOE_OK;
+}
+
+int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t ws_bytes,
+                      void *stream) {
+    Params p;
+    bool decode = false, router = false;
+    const int pr = prepare_forward(h, io, ws, ws_bytes, p, decode, router);
+    if (pr == kNothingToDo) return NVFP4_MOE_OK;
+    if (pr != NVFP4_MOE_OK) return pr;
+    const nvfp4_moe_dims &d = h->d;
+    const int T = io->T;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // External records, so that a forward captured into a CUDA graph records the
     // phase events on every replay (a plain record inside capture is only an
@@ -377,6 +392,41 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
         mark(4);
     }
     return cudaGetLastError() == cudaSuccess ? NVFP4_MOE_OK : NVFP4_MOE_ERR_CUDA;
+}
+
+int nvfp4_moe_forward_decode_stack(nvfp4_moe_t *const *layers, int32_t n_layers, const nvfp4_moe_io *io,
+                                   void *ws, size_t ws_bytes, void *stream) {
+    if (!layers || !io || n_layers < 1 || n_layers > NVFP4_MOE_MAX_STACK) return NVFP4_MOE_ERR_INVALID_ARG;
+    for (int l = 0; l < n_layers; l++) {
+        if (!layers[l]) return NVFP4_MOE_ERR_INVALID_ARG;
+        const nvfp4_moe_dims &a = layers[l]->d, &b0 = layers[0]->d;
+        if (a.hidden != b0.hidden || a.inter != b0.inter || a.n_experts != b0.n_experts ||
+            a.top_k != b0.top_k || layers[l]->device != layers[0]->device)
+            return NVFP4_MOE_ERR_INVALID_ARG;
+        if (io->T > a.max_tokens) return NVFP4_MOE_ERR_INVALID_ARG;
+    }
+    // the residual stream in place, routed from per-layer logits
+    if (io->act_type != NVFP4_MOE_ACT_F32 || io->out_type != NVFP4_MOE_OUT_F32_ADD || io->act != io->out ||
+        !io->router_logits || io->router_w || io->topk_ids || io->topk_weights)
+        return NVFP4_MOE_ERR_INVALID_ARG;
+    if (io->dbg_ids || io->dbg_w || io->dbg_counts || io->dbg_offsets || io->dbg_perm || io->dbg_logits)
+        return NVFP4_MOE_ERR_INVALID_ARG;
+    Params p;
+    bool decode = false, router = false;
+    const int pr = prepare_forward(layers[0], io, ws, ws_bytes, p, decode, router);
+    if (pr == kNothingToDo) return NVFP4_MOE_OK;
+    if (pr != NVFP4_MOE_OK) return pr;
+    if (!decode) return NVFP4_MOE_ERR_UNSUPPORTED_DIMS;
+    DecLayerPtrs w[NVFP4_MOE_MAX_STACK];
+    for (int l = 0; l < n_layers; l++) {
+        const nvfp4_moe_weights &x = layers[l]->w;
+        w[l] = DecLayerPtrs{x.gate_codes, x.up_codes, x.gate_scales, x.up_scales, x.gate_global,
+                            x.up_global, x.down_codes, x.down_scales, x.down_global};
+    }
+    if (launch_decode_stack(p, w, n_layers, io->router_logits, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return NVFP4_MOE_ERR_CUDA;
+    return NVFP4_MOE_OK;
 }
 
 int nvfp4_moe_get_status(nvfp4_moe_t *h, void *stream) {
