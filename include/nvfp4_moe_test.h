@@ -22,6 +22,13 @@ extern "C" {
  * which calls with the flag off are correct again. */
 #define NVFP4_MOE_TEST_DECODE_STALL 1
 
+/* Grouped-GEMM path (T > 8): every used expert takes the tensor-core tiles,
+ * none the small-expert streaming kernels (experts with at most 16 pairs), so
+ * that tests can check both paths on the same inputs. The result agrees with
+ * the default within the documented tolerance, not bit for bit (the two sum K
+ * in a different order). */
+#define NVFP4_MOE_TEST_NO_SMALL 2
+
 /* Sets the test flags of a handle (0 = none). Returns NVFP4_MOE_OK, or
  * NVFP4_MOE_ERR_INVALID_ARG for a NULL handle or an unknown flag. */
 NVFP4_MOE_API int nvfp4_moe_test_set_flags(nvfp4_moe_t *h, int32_t flags);

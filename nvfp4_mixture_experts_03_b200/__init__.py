@@ -34,6 +34,7 @@ EXPORTS = ("nvfp4_moe_create", "nvfp4_moe_workspace_bytes", "nvfp4_moe_forward",
            "nvfp4_moe_forward_decode_static", "nvfp4_moe_forward_decode_stack",
            "nvfp4_moe_test_set_flags", "nvfp4_moe_test_fail_alloc", "nvfp4_moe_test_last_detail")
 TEST_DECODE_STALL = 1   # include/nvfp4_moe_test.h
+TEST_NO_SMALL = 2       # every used expert takes the grouped-GEMM tiles
 PHASE_EVENTS = 5
 
 
@@ -148,7 +149,9 @@ def nvfp4_moe_set_phase_events(handle: int, events) -> int:
 
 def nvfp4_moe_test_set_flags(handle: int, flags: int) -> int:
     """Test hook (include/nvfp4_moe_test.h): TEST_DECODE_STALL makes decode's grid
-    barrier wait run out, so the call latches TIMEOUT."""
+    barrier wait run out, so the call latches TIMEOUT; TEST_NO_SMALL sends every
+    used expert through the grouped-GEMM tiles (none through the small-expert
+    kernels)."""
     return lib().nvfp4_moe_test_set_flags(C.c_void_p(handle), C.c_int32(flags))
 
 

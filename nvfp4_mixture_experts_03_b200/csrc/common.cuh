@@ -29,7 +29,10 @@ constexpr int kDnRows = 256;           // hidden rows per down tile (128 per CTA
 enum : int { kStatusCode = 0, kStatusDetail = 1, kStatusWords = 64 };
 
 // Per-call routing/tile counters kept in the workspace (int32 words).
-enum : int { kCntTilesGu = 0, kCntTilesDn = 1, kCntUniq = 2, kCntWords = 64 };
+enum : int { kCntTilesGu = 0, kCntTilesDn = 1, kCntUniq = 2, kCntSmall = 3, kCntWords = 64 };
+// Experts with at most this many pairs skip the grouped-GEMM tiles and are
+// streamed through mma.sync instead (two 8-token halves of one m16n8k16 pass).
+constexpr int kSmallTok = 16;
 // Decode state (per handle, int32 counters): kDsArrive: CTAs at the grid barrier
 // (zero between launches); kDsGen: barrier generation (counts launches; any
 // value is valid, so the state may be cleared at any time between launches).
@@ -78,6 +81,8 @@ struct Params {
     float *ph;                 // [P] prefill: 2^hexp of the pair's token at each position
     float *phinv;              // [T] prefill: 2^-hexp per token
     Tile *tiles_gu, *tiles_dn;
+    int32_t *small_e;          // [E] prefill: experts with 1..small_tok pairs, ascending
+    int32_t small_tok;         // prefill: pair count up to which an expert is small (0: none)
     __half *xh;                // prefill: [P][H] F16 activations per pair position, then the
                                // down projection's w * s_d * y per pair (F16)
     __half *h;                 // [P][I]
@@ -395,6 +400,10 @@ __device__ inline int h_exp_for(float amax) {
 void launch_route_large(const Params &p, cudaStream_t s);
 void launch_prep_prefill(const Params &p, cudaStream_t s);
 void launch_combine(const Params &p, cudaStream_t s);   // prefill: per-token sum of the K pair rows
+// prefill, experts with <= small_tok pairs: mode 0 gate/up + SwiGLU, mode 1 down
+cudaError_t launch_small(int mode, const Params &p, cudaStream_t s);
+cudaError_t small_init();
+bool small_fits(int H, int I);   // the small-expert kernels' shared memory fits
 cudaError_t launch_decode(const Params &p, cudaStream_t s);   // the whole T <= 8 layer
 // One layer's weight planes, for a decode stack.
 struct DecLayerPtrs {

@@ -43,16 +43,9 @@
 // multiples of 32: a 32-wide piece of a round past the end is zero on both sides.
 #include "common.cuh"
 #include "route_common.cuh"
+#include "stream_common.cuh"
 
 namespace nvmoe {
-
-__device__ inline uint4 ldg_stream(const void *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
 
 __device__ inline void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ inline void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
@@ -379,21 +372,6 @@ __device__ inline void store_out(const Params &p, int rb, const float4 &v, int g
     }
 }
 
-// Latches NONFINITE (detail: stage | expert or row) if any lane of the warp saw
-// a bad value.
-__device__ inline void warp_report(const Params &p, int bad, int stage) {
-    const unsigned m = __ballot_sync(0xffffffffu, bad >= 0);
-    if (m) {
-        const int v = __shfl_sync(0xffffffffu, bad, __ffs(m) - 1);
-        if ((threadIdx.x & 31) == 0) latch_status(p.status, NVFP4_MOE_ERR_NONFINITE, stage | v);
-    }
-}
-
-__device__ inline void cp_async16(void *smem, const void *gmem) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
-                 : "memory");
-}
-
 // Bounded wait until *word != old (one thread); latches TIMEOUT on give-up.
 __device__ inline bool wait_ne(const int32_t *word, int old, int32_t *status, int where) {
     const volatile int32_t *v = word;
@@ -418,13 +396,6 @@ __host__ __device__ inline size_t dec_xs_bytes(int T, int H) {
     return ((size_t)(T + 1) * dec_ld1(H) * 2 + 15) & ~(size_t)15;
 }
 __host__ __device__ inline int dec_ld2(int I) { return cdiv(I, 128) * 128 + 8; }
-
-// [a, b) = worker w's share of n units when W workers split them evenly in
-// contiguous ranges.
-__device__ inline void share(int n, int w, int W, int &a, int &b) {
-    a = (int)((long long)n * w / W);
-    b = (int)((long long)n * (w + 1) / W);
-}
 
 // The warp (of W) whose share of n units holds unit x.
 __device__ inline int owner(int n, int W, int x) {

@@ -105,7 +105,7 @@ bool use_decode(const nvfp4_moe_dims &d, int T) {
 
 struct WsLayout {
     size_t cnt, ids, wts, hist, cbase, counts, offsets, perm, inv, ptok, pw, ps, xscale, ph, phinv, tiles_gu,
-        tiles_dn, xh, h, rlogits, total;
+        tiles_dn, small_e, xh, h, rlogits, total;
     int nch, max_gu, max_dn;
 };
 
@@ -141,6 +141,7 @@ WsLayout layout(const nvfp4_moe_dims &d, int T) {
     L.phinv = take(decode ? 0 : (size_t)T * 4);
     L.tiles_gu = take((size_t)L.max_gu * sizeof(Tile));
     L.tiles_dn = take((size_t)L.max_dn * sizeof(Tile));
+    L.small_e = take(decode ? 0 : (size_t)E * 4);
     L.xh = take(decode ? 0 : P * d.hidden * 2);   // decode stages activations in shared memory
     L.h = take(P * d.inter * 2);
     L.rlogits = take((size_t)T * E * 4);   // router projection output (when used)
@@ -201,7 +202,7 @@ int nvfp4_moe_create(nvfp4_moe_t **out, const nvfp4_moe_dims *dims,
     if (major != 10) return NVFP4_MOE_ERR_NO_DEVICE;
     int pf_clusters = 0;
     if (prefill_init(&pf_clusters) != cudaSuccess || decode_init() != cudaSuccess ||
-        router_init() != cudaSuccess || !encode_fn())
+        router_init() != cudaSuccess || small_init() != cudaSuccess || !encode_fn())
         return NVFP4_MOE_ERR_CUDA;
     nvfp4_moe *h = new (std::nothrow) nvfp4_moe;
     if (!h) return NVFP4_MOE_ERR_CUDA;
@@ -318,6 +319,8 @@ static int prepare_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, siz
     p.phinv = reinterpret_cast<float *>(b + L.phinv);
     p.tiles_gu = reinterpret_cast<Tile *>(b + L.tiles_gu);
     p.tiles_dn = reinterpret_cast<Tile *>(b + L.tiles_dn);
+    p.small_e = reinterpret_cast<int32_t *>(b + L.small_e);
+    p.small_tok = (h->test_flags & NVFP4_MOE_TEST_NO_SMALL) || !small_fits(d.hidden, d.inter) ? 0 : kSmallTok;
     p.xh = reinterpret_cast<__half *>(b + L.xh);
     p.h = reinterpret_cast<__half *>(b + L.h);
     p.status = h->status;
@@ -383,10 +386,12 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
         mark(1);
         launch_prep_prefill(p, s);
         mark(2);
-        if (launch_prefill_gemm(0, p, map_xh, h->codes, h->pf_clusters, s) != cudaSuccess)
+        if (launch_prefill_gemm(0, p, map_xh, h->codes, h->pf_clusters, s) != cudaSuccess ||
+            launch_small(0, p, s) != cudaSuccess)
             return NVFP4_MOE_ERR_CUDA;
         mark(3);
-        if (launch_prefill_gemm(1, p, map_h, h->codes, h->pf_clusters, s) != cudaSuccess)
+        if (launch_prefill_gemm(1, p, map_h, h->codes, h->pf_clusters, s) != cudaSuccess ||
+            launch_small(1, p, s) != cudaSuccess)
             return NVFP4_MOE_ERR_CUDA;
         launch_combine(p, s);
         mark(4);
@@ -459,7 +464,7 @@ int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events, int32_t n_ev
 }
 
 int nvfp4_moe_test_set_flags(nvfp4_moe_t *h, int32_t flags) {
-    if (!h || (flags & ~NVFP4_MOE_TEST_DECODE_STALL)) return NVFP4_MOE_ERR_INVALID_ARG;
+    if (!h || (flags & ~(NVFP4_MOE_TEST_DECODE_STALL | NVFP4_MOE_TEST_NO_SMALL))) return NVFP4_MOE_ERR_INVALID_ARG;
     h->test_flags = flags;
     return NVFP4_MOE_OK;
 }

@@ -95,37 +95,45 @@ __global__ void __launch_bounds__(1024) route_chunkscan_kernel(Params p) {
     if (lane == 0) p.counts[e] = carry;
 }
 
-// Kernel 3 (one CTA of 1024 threads): expert offsets and the grouped-GEMM tile
-// lists.
+// Kernel 3 (one CTA of 1024 threads): expert offsets, the grouped-GEMM tile
+// lists (experts with more than small_tok pairs) and the list of small experts.
 __global__ void __launch_bounds__(1024) route_scan_kernel(Params p) {
     extern __shared__ int sm[];
     int *cnt_s = sm;                      // [E]
     int *off_s = cnt_s + p.E;             // [E+1]
     int *gub = off_s + p.E + 1;           // [E]
     int *dnb = gub + p.E;                 // [E]
-    int *wt = dnb + p.E;                  // [33]
+    int *sml = dnb + p.E;                 // [E]
+    int *wt = sml + p.E;                  // [33]
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) cnt_s[e] = p.counts[e];
     __syncthreads();
     const int mgu = cdiv(p.I, kGuRows), mdn = cdiv(p.H, kDnRows);
+    auto small = [&](int c) { return c > 0 && c <= p.small_tok; };
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
-        off_s[e] = cnt_s[e];
-        gub[e] = cdiv(cnt_s[e], kBN) * mgu;
-        dnb[e] = cdiv(cnt_s[e], kBN) * mdn;
+        const int c = cnt_s[e];
+        const int nt = small(c) ? 0 : cdiv(c, kBN);
+        off_s[e] = c;
+        gub[e] = nt * mgu;
+        dnb[e] = nt * mdn;
+        sml[e] = small(c) ? 1 : 0;
     }
     __syncthreads();
     const int total = block_exscan(off_s, p.E, wt);
     const int ngu = block_exscan(gub, p.E, wt);
     const int ndn = block_exscan(dnb, p.E, wt);
+    const int nsm = block_exscan(sml, p.E, wt);
     if (threadIdx.x == 0) {
         off_s[p.E] = total;
         p.cnt[kCntTilesGu] = ngu;
         p.cnt[kCntTilesDn] = ndn;
+        p.cnt[kCntSmall] = nsm;
     }
     __syncthreads();
     for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
         p.offsets[e] = off_s[e];
         if (p.dbg_offsets) p.dbg_offsets[e] = off_s[e];
         if (e < p.E && p.dbg_counts) p.dbg_counts[e] = cnt_s[e];
+        if (e < p.E && small(cnt_s[e])) p.small_e[sml[e]] = e;
     }
     for (int slot = threadIdx.x; slot < ngu; slot += blockDim.x)
         emit_tile(p.tiles_gu, gub, cnt_s, off_s, p.E, mgu, kGuRows, slot);
@@ -299,7 +307,7 @@ void launch_route_large(const Params &p, cudaStream_t s) {
     const size_t mask_bytes = 2 * p.E * sizeof(uint32_t);
     NPER_SWITCH(p.E, (route_topk_hist_kernel<NP><<<p.nch, topk_threads<NP>(), mask_bytes, s>>>(p)));
     route_chunkscan_kernel<<<cdiv(p.E, 32), 1024, 0, s>>>(p);
-    const size_t scan_bytes = (4 * p.E + 1 + 33) * sizeof(int);
+    const size_t scan_bytes = (5 * p.E + 1 + 33) * sizeof(int);
     route_scan_kernel<<<1, 1024, scan_bytes, s>>>(p);
     route_scatter_kernel<<<p.nch, 256, mask_bytes, s>>>(p);
 }

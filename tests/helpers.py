@@ -35,12 +35,15 @@ def assert_close(got, ref, what=""):
 
 
 def run_gpu(layer_gpu, x, *, K, logits=None, ids=None, wts=None, x_scale=None, max_tokens=None,
-            out=None, accumulate=False):
-    """Runs the CUDA layer with debug routing outputs; returns (out, debug dict, status)."""
+            out=None, accumulate=False, flags=0):
+    """Runs the CUDA layer with debug routing outputs; returns (out, debug dict, status).
+    `flags`: test flags of include/nvfp4_moe_test.h set on the handle first."""
     import nvfp4_mixture_experts_03_b200 as nv
     T = x.shape[0]
     E = layer_gpu.dims.E
     m = nv.MoELayer.from_layer(layer_gpu, top_k=K, max_tokens=max_tokens or max(T, 1))
+    if flags:
+        assert nv.nvfp4_moe_test_set_flags(m.handle, flags) == 0
     dbg = nv.debug_buffers(T, E, K, x.device)
     o = m.forward(x, logits=logits, topk_ids=ids, topk_weights=wts, x_scale=x_scale, out=out,
                   accumulate=accumulate, debug=dbg)

@@ -25,6 +25,9 @@ def _case(dims, T, seed, *, zipf=None, act="bf16", outliers=False):
     return layer, logits, x, xs
 
 
+NO_SMALL = 2   # include/nvfp4_moe_test.h: NVFP4_MOE_TEST_NO_SMALL
+
+
 def _run_both(layer, logits, x, xs, K, **kw):
     ref = oracle.forward(layer, x, K=K, logits=logits, x_scale=xs)
     lg = layer.to(DEV)
@@ -189,14 +192,16 @@ def _scaled(layer, **factors):
     return synth.Layer(layer.dims, **kw)
 
 
-@pytest.mark.parametrize("T", [4, 64])
+@pytest.mark.parametrize("T", [4, 12, 64])
 @pytest.mark.parametrize("which", ["down", "gate_up"])
 def test_f16_range_overflow_is_reported_never_silent(T, which):
     """Globals scaled by powers of two push the F16 intermediates past 65504: the
     down global pushes the grouped-GEMM path's per-pair rows w*s_d*y out of range
     (decode keeps y in FP32), the gate and up globals push h out of range on both
     paths. The result must be either correct (FP32 math kept it in range) or
-    flagged NVFP4_MOE_ERR_NONFINITE -- never a silent inf in the output."""
+    flagged NVFP4_MOE_ERR_NONFINITE -- never a silent inf in the output. T = 12
+    leaves every expert with at most 16 pairs (the small-expert kernels), T = 64
+    sends most of them through the tensor-core tiles."""
     dims = synth.TINY
     base, logits, x, _ = _case(dims, T, seed=63)
     if which == "down":
@@ -234,9 +239,9 @@ def test_outputs_are_bitwise_reproducible(T):
     assert torch.equal(a.view(torch.int32), b.view(torch.int32))
 
 
-@pytest.mark.parametrize("T", [5, 70])
+@pytest.mark.parametrize("T,flags", [(5, 0), (70, 0), (70, NO_SMALL), (20, 0)])
 @pytest.mark.parametrize("H,I", [(160, 96), (224, 160), (256, 96), (160, 256), (96, 288)])
-def test_hidden_and_inter_multiples_of_32(H, I, T):
+def test_hidden_and_inter_multiples_of_32(H, I, T, flags):
     """H and I that are multiples of 32 but not of 128: K rounds and K steps with a
     zero-padded tail, partial gate/up and down row tiles, and scale rows that are
     not 8-byte aligned. The last expert is made popular so the partial tiles at
@@ -244,8 +249,30 @@ def test_hidden_and_inter_multiples_of_32(H, I, T):
     dims = synth.LayerDims(E=6, H=H, I=I, K=2)
     layer, logits, x, xs = _case(dims, T, seed=81 + H + I)
     logits[:, dims.E - 1] += 1.5
-    ref, out, dbg, st = _run_both(layer, logits, x, xs, dims.K)
+    ref, out, dbg, st = _run_both(layer, logits, x, xs, dims.K, flags=flags)
     assert st == 0
     assert ref["counts"][dims.E - 1] > 0
     check_routing(dbg, ref, T, dims.K)
-    assert_close(out, ref["out"], f"H={H} I={I} T={T}")
+    assert_close(out, ref["out"], f"H={H} I={I} T={T} flags={flags}")
+
+
+@pytest.mark.parametrize("flags", [0, NO_SMALL])
+@pytest.mark.parametrize("T", [24, 90, 700])
+def test_small_experts_and_tiles(T, flags):
+    """64 experts: at T = 24 (uniform routing) every expert has at most 16 pairs
+    (all take the small-expert kernels); with Zipf-skewed routing at T = 90 the
+    hot experts take the tensor-core tiles and the tail the small-expert kernels,
+    at T = 700 most take the tiles. With NVFP4_MOE_TEST_NO_SMALL every expert
+    takes the tiles. Every combination against the oracle."""
+    dims = synth.LayerDims(E=64, H=512, I=384, K=6)
+    layer, logits, x, xs = _case(dims, T, seed=91 + T, zipf=None if T == 24 else 1.1, outliers=True)
+    ref, out, dbg, st = _run_both(layer, logits, x, xs, dims.K, flags=flags)
+    assert st == 0
+    check_routing(dbg, ref, T, dims.K)
+    c = ref["counts"]
+    small = int(((c > 0) & (c <= 16)).sum())
+    if T == 24:
+        assert c.max() <= 16
+    else:
+        assert small > 0 and c.max() > 16
+    assert_close(out, ref["out"], f"small/tiles T={T} flags={flags}")
