@@ -259,10 +259,17 @@ def run_ours(args, ws, rank, local):
     # step (sw_power_cap is flagged but barely lowers it), so the burst cuBLAS figure
     # is the denominator; the sustained one is context.
     peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    traffic = profile_traffic("grouped_gemm_gateup", wl.name)
-    roof = {"kernel": "grouped_gemm_kernel<0> (gate/up + SwiGLU)", "bound": "tensor",
+    # The gate/up phase is two launches: the tensor-core tiles of the experts with
+    # more than 16 pairs and the streaming kernel of the rest; its traffic is the
+    # sum of both captures (None unless both match the current sources).
+    t_tiles = profile_traffic("grouped_gemm_gateup", wl.name)
+    t_small = profile_traffic("small_expert_gateup", wl.name)
+    traffic = t_tiles + t_small if t_tiles is not None and t_small is not None else None
+    roof = {"kernel": "gate/up + SwiGLU phase: grouped_gemm_kernel<0> (tensor-core tiles) + "
+                      "small_expert_kernel<0> (experts with <= 16 pairs)", "bound": "tensor",
             "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4), "traffic": traffic,
+            "traffic_parts": {"grouped_gemm_kernel<0>": t_tiles, "small_expert_kernel<0>": t_small},
             "peak_source": f"{pk_src} bf16_tflops, burst (F16 operands run at the BF16 rate); "
                            f"sustained {pk.get('bf16_tflops_sustained')} for context",
             "frac_of_sustained": round(achieved / pk.get("bf16_tflops_sustained",

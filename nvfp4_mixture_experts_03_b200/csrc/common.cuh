@@ -29,7 +29,8 @@ constexpr int kDnRows = 256;           // hidden rows per down tile (128 per CTA
 enum : int { kStatusCode = 0, kStatusDetail = 1, kStatusWords = 64 };
 
 // Per-call routing/tile counters kept in the workspace (int32 words).
-enum : int { kCntTilesGu = 0, kCntTilesDn = 1, kCntUniq = 2, kCntSmall = 3, kCntWords = 64 };
+// kCntSmallQ, +1: the small-expert kernels' item queues (gate/up, down).
+enum : int { kCntTilesGu = 0, kCntTilesDn = 1, kCntUniq = 2, kCntSmall = 3, kCntSmallQ = 4, kCntWords = 64 };
 // Experts with at most this many pairs skip the grouped-GEMM tiles and are
 // streamed through mma.sync instead (two 8-token halves of one m16n8k16 pass).
 constexpr int kSmallTok = 16;
@@ -118,6 +119,11 @@ __device__ inline bool fits_f16(float x) { return fabsf(x) < 65520.0f; }
 __device__ inline uint32_t smem_u32(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
+
+// Programmatic dependent launch: wait for the grid this one depends on (its
+// writes visible); let the grid that depends on this one start launching.
+__device__ inline void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ inline void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
 __device__ inline uint64_t globaltimer() {
     uint64_t t;

@@ -47,8 +47,6 @@
 
 namespace nvmoe {
 
-__device__ inline void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ inline void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
 // Eight mma steps of one 128-wide K round: A rows (g: ca, g+8: cb) as 16 code
 // bytes each with their two group scales; B from `bfrag(s)`.

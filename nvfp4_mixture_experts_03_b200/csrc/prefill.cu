@@ -216,6 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *colu_s = colf_s + kBN;                 // gate/up: the up factor (see the epilogue)
     Bars *bars = reinterpret_cast<Bars *>(epi_stage + kEpiBytes + 2 * kColBytes);
     volatile int *abort = &bars->abort;
+    // The small-expert kernel that follows on the stream reads nothing this grid
+    // writes: it may take the SMs this grid leaves while its last tiles run.
+    grid_dep_launch();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)cluster_ctarank();

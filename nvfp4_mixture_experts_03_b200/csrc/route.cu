@@ -127,6 +127,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(Params p) {
         p.cnt[kCntTilesGu] = ngu;
         p.cnt[kCntTilesDn] = ndn;
         p.cnt[kCntSmall] = nsm;
+        p.cnt[kCntSmallQ] = 0;
+        p.cnt[kCntSmallQ + 1] = 0;
     }
     __syncthreads();
     for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {

@@ -14,12 +14,16 @@
 //
 // Work: the list of small experts (ascending, built with the tile lists) times
 // S pieces per expert (S chosen on the device from the list's length and the
-// grid, the same in every CTA) gives the items; CTA b takes items b, b + grid,
-// ... For each item the CTA stages the expert's pair rows (activations for
-// gate/up, h for down) in shared memory with a zero row for absent pairs, and
-// its 16 warps split the item's granules (gate/up: 8 intermediates, gate and up
-// rows; down: 16 hidden rows) in contiguous ranges, every granule whole in one
-// warp, so each output is summed in a fixed order and written once.
+// grid, the same in every CTA) gives the items, which the CTAs take from a
+// queue (one atomic per item). Each kernel is launched as a programmatic
+// dependent of the tile kernel before it, which lets it start at once: its
+// CTAs take the SMs the tile kernel's CTAs leave as they finish, and a CTA that
+// starts late finds fewer items left. For each item the CTA stages the expert's
+// pair rows (activations for gate/up, h for down) in shared memory with a zero
+// row for absent pairs, and its 16 warps split the item's granules (gate/up: 8
+// intermediates, gate and up rows; down: 16 hidden rows) in contiguous ranges,
+// every granule whole in one warp, so each output is summed in a fixed order
+// and written once, whichever CTA takes the item.
 //
 // Outputs match the tile kernels': gate/up stores h = silu(g) * u (F16, times
 // the token's 2^hexp) at the pair's row of h; down stores y * s_d * w (F16) at
@@ -175,20 +179,14 @@ __device__ inline void se_round(float (&acc0)[4], float (&acc1)[4], const uint4 
     }
 }
 
-// Pieces per expert for nse experts of `units` granules on G CTAs: fewest item
-// waves times the largest per-warp share (plus one for the staging of each
-// item); among equal costs the most pieces (more SMs streaming).
+// Pieces per expert for nse experts of `units` granules on G CTAs: about two
+// items per CTA (a CTA that starts late, or whose items run long, leaves the
+// rest to the others), at most one piece per 16 granules (a granule for every
+// warp) and at least one.
 __device__ inline int se_pieces(int nse, int units, int G) {
-    int best = 1;
-    long long bc = -1;
-    for (int S = 1; S <= units && S <= kSeMaxPieces; S++) {
-        const long long c = (long long)cdiv(nse * S, G) * (cdiv(cdiv(units, S), kSeWarps) + 1);
-        if (bc < 0 || c <= bc) {
-            bc = c;
-            best = S;
-        }
-    }
-    return best;
+    if (nse <= 0) return 1;
+    const int want = cdiv(2 * G, nse), most = max(1, units / kSeWarps);
+    return max(1, min(min(want, most), kSeMaxPieces));
 }
 
 // Copies the n pair rows (K F16 each, row stride K in global, se_ld here, pieces
@@ -209,8 +207,8 @@ template <int MODE>
 __global__ void __launch_bounds__(kSeThreads, 1) small_expert_kernel(Params p) {
     constexpr int NR = MODE == 0 ? kSeGuRounds : kSeDnRounds;
     extern __shared__ __align__(16) uint8_t se_sm[];
+    __shared__ int s_item;
     const int nse = p.cnt[kCntSmall];
-    if (nse == 0) return;
     const int H = p.H, I = p.I;
     const int Kin = MODE == 0 ? H : I;              // length of a staged row
     const int C = se_chunks(Kin, NR);               // chunks per weight row
@@ -227,12 +225,18 @@ __global__ void __launch_bounds__(kSeThreads, 1) small_expert_kernel(Params p) {
     const uint8_t *cbase_b = MODE == 0 ? p.up_codes : p.down_codes;
     const bool v32 = kb % 32 == 0 && ((uintptr_t)cbase_a | (uintptr_t)cbase_b) % 32 == 0;
     const int S = se_pieces(nse, units, gridDim.x);
-    {
+    if (nse > 0) {
         uint4 *z = reinterpret_cast<uint4 *>(se_sm);
         for (size_t i = threadIdx.x; i < se_smem(Kin, NR) / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
     }
     int bad = -1;
-    for (int it = blockIdx.x; it < nse * S; it += gridDim.x) {
+    for (;;) {
+        // the next item; the barrier also ends every warp's use of the previous
+        // item's rows and factors
+        if (threadIdx.x == 0) s_item = atomicAdd(p.cnt + kCntSmallQ + MODE, 1);
+        __syncthreads();
+        const int it = s_item;
+        if (it >= nse * S) break;
         const int u = it / S, piece = it - u * S;
         const int e = p.small_e[u], n = p.counts[e], pos0 = p.offsets[e];
         int ia, ib, wa, wb;
@@ -265,7 +269,6 @@ __global__ void __launch_bounds__(kSeThreads, 1) small_expert_kernel(Params p) {
         SeBuf<NR> b0, b1, b2;
         if (x < end) issue(b0);   // in flight while the rows are staged
         if (x + 1 < end) issue(b1);
-        __syncthreads();   // every warp is done with the previous item's rows and factors
         se_stage<NR>(xs, (MODE == 0 ? p.xh + (size_t)pos0 * H : p.h + (size_t)pos0 * I), n, Kin);
         if (threadIdx.x < kSmallTok) {
             // epilogue factors of pair slot t: gate/up: s_g * x's staging factor and
@@ -342,31 +345,43 @@ __global__ void __launch_bounds__(kSeThreads, 1) small_expert_kernel(Params p) {
         }
     }
     warp_report(p, bad, MODE == 0 ? kNfH : kNfY);
+    // complete only after the tile kernel this grid was launched behind, so that
+    // the launches after it on the stream see both grids' outputs
+    grid_dep_wait();
 }
 
 int sm_count();   // SMs of the current device (decode.cu)
 
+// Shared memory a small-expert kernel may take (the dynamic part; the kernel
+// also has a few bytes of static shared memory).
+constexpr int kSeSmemMax = 200 * 1024;
+
 cudaError_t small_init() {
-    const int bytes = 227 * 1024;
-    cudaError_t e = cudaFuncSetAttribute(small_expert_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaError_t e = cudaFuncSetAttribute(small_expert_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSeSmemMax);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(small_expert_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        e = cudaFuncSetAttribute(small_expert_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSeSmemMax);
     return e;
 }
 
 // Whether the small-expert path fits shared memory for these dimensions.
 bool small_fits(int H, int I) {
-    return se_smem(H, kSeGuRounds) <= 227 * 1024 && se_smem(I, kSeDnRounds) <= 227 * 1024;
+    return se_smem(H, kSeGuRounds) <= kSeSmemMax && se_smem(I, kSeDnRounds) <= kSeSmemMax;
 }
 
 cudaError_t launch_small(int mode, const Params &p, cudaStream_t s) {
     if (p.small_tok <= 0) return cudaSuccess;
-    const size_t bytes = mode == 0 ? se_smem(p.H, kSeGuRounds) : se_smem(p.I, kSeDnRounds);
-    if (mode == 0)
-        small_expert_kernel<0><<<sm_count(), kSeThreads, bytes, s>>>(p);
-    else
-        small_expert_kernel<1><<<sm_count(), kSeThreads, bytes, s>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sm_count());
+    cfg.blockDim = dim3(kSeThreads);
+    cfg.dynamicSmemBytes = mode == 0 ? se_smem(p.H, kSeGuRounds) : se_smem(p.I, kSeDnRounds);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return mode == 0 ? cudaLaunchKernelEx(&cfg, small_expert_kernel<0>, p)
+                     : cudaLaunchKernelEx(&cfg, small_expert_kernel<1>, p);
 }
 
 }  // namespace nvmoe
