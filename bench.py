@@ -755,7 +755,7 @@ def main():
         res = run_ours(args, ws, rank, local)
         # The default single-GPU run also carries the other two timed configurations
         # as sub-records: the 32768-token W4A8 chunk and the 48-layer stack.
-        if args.workload == "prefill8k" and ws == 1 and not args.no_subrecords:
+        if args.workload == "prefill8k" and ws == 1 and not args.no_subrecords and not args.decode_only:
             torch.cuda.empty_cache()
             sub = argparse.Namespace(**vars(args))
             sub.workload, sub.no_decode, sub.steps = "w4a8_32k", True, max(5, min(args.steps, 40))

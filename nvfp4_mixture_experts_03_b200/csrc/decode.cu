@@ -227,11 +227,15 @@ struct DecStack {
 };
 
 // Gate/up weights of one warp's chunk: rows g (gate) and g+8 (up), up to
-// kGuRounds rounds.
+// kGuRounds rounds. Scales: per round, row g's two scale bytes in bits 0..15 of
+// s[j] and row g+8's in 16..31; or, when whole 8-byte scale pieces can be read
+// (gu_issue's `vec`), round r0 + q's eight bytes of row g in s[0..1] and of row
+// g+8 in s[2..3], which gu_scales hands to the four lanes of the quad.
 struct GuBuf {
     uint4 ca[kGuRounds], cb[kGuRounds];
-    uint32_t s[kGuRounds];   // row g's two scale bytes in bits 0..15, row g+8's in 16..31
+    uint32_t s[kGuRounds];
 };
+static_assert(kGuRounds == 4, "a quad's four lanes fetch the scale pieces of a chunk's four rounds");
 
 // A run of at most kGuRounds consecutive K rounds of one granule (CTA-local).
 struct Chunk {
@@ -252,14 +256,25 @@ __device__ inline Chunk take_chunk(int &x, int end, int R) {
 
 // Weight loads of rounds [c.r0, c.r1) of granule P.gb + c.item; 16-byte pieces
 // past the row's end (H not a multiple of 128) are zero, with zero scales.
+// `vec` (H a multiple of 128, 8-byte aligned scale planes): lane q of the quad
+// fetches round c.r0 + q's eight scale bytes of both rows in one load each,
+// instead of every lane fetching two bytes of every round.
 __device__ inline void gu_issue(const Params &p, const DecLayer &W, const DecRoute &R, const DecPlan &P,
-                                const Chunk &c, int g, int q, GuBuf &b) {
+                                const Chunk &c, int g, int q, bool vec, GuBuf &b) {
     if (c.r1 == 0) return;
     const int per_u = p.I / 8, gi = P.gb + c.item, u = gi / per_u;
     const size_t ra = (size_t)R.uniq[u] * p.I + (gi - u * per_u) * 8 + g;
     const int kb = p.H / 2;
     const uint8_t *ca_p = W.gate_codes + ra * kb, *cb_p = W.up_codes + ra * kb;
     const uint8_t *sa_p = W.gate_scales + ra * (p.H / 16), *sb_p = W.up_scales + ra * (p.H / 16);
+    if (vec && c.r0 + q < c.r1) {
+        const uint2 va = __ldg(reinterpret_cast<const uint2 *>(sa_p + 8 * (c.r0 + q)));
+        const uint2 vb = __ldg(reinterpret_cast<const uint2 *>(sb_p + 8 * (c.r0 + q)));
+        b.s[0] = va.x;
+        b.s[1] = va.y;
+        b.s[2] = vb.x;
+        b.s[3] = vb.y;
+    }
 #pragma unroll
     for (int j = 0; j < kGuRounds; j++) {
         const int r = c.r0 + j;
@@ -267,14 +282,28 @@ __device__ inline void gu_issue(const Params &p, const DecLayer &W, const DecRou
             if (64 * r + 16 * q < kb) {
                 b.ca[j] = ldg_stream(ca_p + 64 * r + 16 * q);
                 b.cb[j] = ldg_stream(cb_p + 64 * r + 16 * q);
-                b.s[j] = (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sa_p + 8 * r + 2 * q)) |
-                         ((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sb_p + 8 * r + 2 * q)) << 16);
+                if (!vec)
+                    b.s[j] = (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sa_p + 8 * r + 2 * q)) |
+                             ((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sb_p + 8 * r + 2 * q)) << 16);
             } else {
                 b.ca[j] = b.cb[j] = make_uint4(0, 0, 0, 0);
                 b.s[j] = 0;
             }
         }
     }
+}
+
+// Round j's scale bytes of this lane (row g in bits 0..15, row g+8 in 16..31)
+// from a chunk loaded with gu_issue's `vec`: lane j of the quad holds round
+// r0 + j's eight bytes of each row; this lane (q) takes bytes 2q and 2q + 1.
+// Every lane of the warp calls it (shuffles).
+__device__ inline uint32_t gu_scales(const GuBuf &b, int j, int lane, int q) {
+    const int src = (lane & ~3) | j;
+    const uint32_t a0 = __shfl_sync(0xffffffffu, b.s[0], src), a1 = __shfl_sync(0xffffffffu, b.s[1], src);
+    const uint32_t b0 = __shfl_sync(0xffffffffu, b.s[2], src), b1 = __shfl_sync(0xffffffffu, b.s[3], src);
+    const int sh = 16 * (q & 1);
+    const uint32_t sa = ((q >> 1) ? a1 : a0) >> sh, sb = ((q >> 1) ? b1 : b0) >> sh;
+    return (sa & 0xFFFFu) | (sb << 16);
 }
 
 // h of granule P.gb + j for this thread's intermediate (row g) and token slots
@@ -511,6 +540,7 @@ __device__ __forceinline__ void decode_body(const Params &p, const DecLayer &W, 
     // this warp's gate/up share; its first loads go out before the activations
     // are staged
     const int R1 = cdiv(H, 128), R2 = cdiv(I, 128);
+    const bool gvec = H % 128 == 0 && ((uintptr_t)W.gate_scales | (uintptr_t)W.up_scales) % 8 == 0;
     const int n1 = (ge - gb) * R1;
     int a1, b1;
     share(n1, warp, kDecWarps, a1, b1);
@@ -519,7 +549,7 @@ __device__ __forceinline__ void decode_body(const Params &p, const DecLayer &W, 
     GuBuf buf0, buf1;
     {
         const DecPlan Pl{gb, ge, 0, 0};
-        gu_issue(p, W, R, Pl, cur, g, q, buf0);
+        gu_issue(p, W, R, Pl, cur, g, q, gvec, buf0);
     }
 
     __syncthreads();   // P is read by every warp from here on
@@ -535,13 +565,14 @@ __device__ __forceinline__ void decode_body(const Params &p, const DecLayer &W, 
         const __half *xrow = xs + (size_t)(g < T ? g : T) * ld1 + 32 * q;
         auto step = [&](GuBuf &b, GuBuf &nb) {
             const Chunk nxt = take_chunk(x1, b1, R1);
-            gu_issue(p, W, R, P, nxt, g, q, nb);
+            gu_issue(p, W, R, P, nxt, g, q, gvec, nb);
 #pragma unroll
             for (int j = 0; j < kGuRounds; j++) {
                 const int r = cur.r0 + j;
                 if (r < cur.r1) {
                     const __half *xr = xrow + 128 * r;
-                    round_mma(acc, b.ca[j], b.cb[j], b.s[j] & 0xFFFF, b.s[j] >> 16,
+                    const uint32_t sj = gvec ? gu_scales(b, j, lane, q) : b.s[j];
+                    round_mma(acc, b.ca[j], b.cb[j], sj & 0xFFFF, sj >> 16,
                               [&](int s, uint32_t &v0, uint32_t &v1) {
                                   const uint2 v = *reinterpret_cast<const uint2 *>(xr + 4 * s);
                                   v0 = v.x;
