@@ -267,13 +267,24 @@ __device__ inline void gu_issue(const Params &p, const DecLayer &W, const DecRou
     const int kb = p.H / 2;
     const uint8_t *ca_p = W.gate_codes + ra * kb, *cb_p = W.up_codes + ra * kb;
     const uint8_t *sa_p = W.gate_scales + ra * (p.H / 16), *sb_p = W.up_scales + ra * (p.H / 16);
-    if (vec && c.r0 + q < c.r1) {
-        const uint2 va = __ldg(reinterpret_cast<const uint2 *>(sa_p + 8 * (c.r0 + q)));
-        const uint2 vb = __ldg(reinterpret_cast<const uint2 *>(sb_p + 8 * (c.r0 + q)));
+    if (vec) {
+        // Every piece lies inside its row, so every load is unconditional (rounds
+        // past c.r1 repeat round c.r1 - 1, unused): each lands straight in its
+        // buffer register, with no select that would wait for it here.
+        const int rq = min(c.r0 + q, c.r1 - 1);
+        const uint2 va = __ldg(reinterpret_cast<const uint2 *>(sa_p + 8 * rq));
+        const uint2 vb = __ldg(reinterpret_cast<const uint2 *>(sb_p + 8 * rq));
         b.s[0] = va.x;
         b.s[1] = va.y;
         b.s[2] = vb.x;
         b.s[3] = vb.y;
+#pragma unroll
+        for (int j = 0; j < kGuRounds; j++) {
+            const int r = min(c.r0 + j, c.r1 - 1);
+            b.ca[j] = ldg_stream(ca_p + 64 * r + 16 * q);
+            b.cb[j] = ldg_stream(cb_p + 64 * r + 16 * q);
+        }
+        return;
     }
 #pragma unroll
     for (int j = 0; j < kGuRounds; j++) {
@@ -282,9 +293,8 @@ __device__ inline void gu_issue(const Params &p, const DecLayer &W, const DecRou
             if (64 * r + 16 * q < kb) {
                 b.ca[j] = ldg_stream(ca_p + 64 * r + 16 * q);
                 b.cb[j] = ldg_stream(cb_p + 64 * r + 16 * q);
-                if (!vec)
-                    b.s[j] = (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sa_p + 8 * r + 2 * q)) |
-                             ((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sb_p + 8 * r + 2 * q)) << 16);
+                b.s[j] = (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sa_p + 8 * r + 2 * q)) |
+                         ((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sb_p + 8 * r + 2 * q)) << 16);
             } else {
                 b.ca[j] = b.cb[j] = make_uint4(0, 0, 0, 0);
                 b.s[j] = 0;
@@ -330,9 +340,11 @@ __device__ inline void swiglu_store(const Params &p, const DecRoute &R, const De
 
 // Down weights of one warp's chunk: kDnUnits units (16-row block, used expert,
 // 128-wide K round), rows g and g+8, 16 code bytes and two scale bytes each.
+// The two scale bytes of each row stay in their own registers as loaded: a
+// combining instruction at issue time would wait there for the loads to land.
 struct DnBuf {
     uint4 ca[kDnUnits], cb[kDnUnits];
-    uint32_t s[kDnUnits];   // as in GuBuf
+    uint32_t sa[kDnUnits], sb[kDnUnits];   // rows g and g+8: two scale bytes each
 };
 
 // Position of a down unit of the CTA (row blocks rb0.., U experts, R2 rounds
@@ -362,8 +374,26 @@ __device__ inline void dn_next(DnCur &c, int U, int R2) {
 // Loads of the n <= kDnUnits down units from c on; 16-byte pieces past the row's
 // end (I not a multiple of 128) are zero, with zero scales.
 __device__ inline void dn_issue(const Params &p, const DecLayer &W, const DecRoute &R, int rb0, DnCur c,
-                                int n, int g, int q, DnBuf &b) {
+                                int n, int g, int q, bool full, DnBuf &b) {
     const int H = p.H, I = p.I, R2 = cdiv(I, 128), U = R.U;
+    if (full) {
+        if (n <= 0) return;
+        // I a multiple of 128: every piece lies inside its row and every load is
+        // unconditional (units past n repeat unit n - 1, unused), landing straight
+        // in its buffer register
+#pragma unroll
+        for (int j = 0; j < kDnUnits; j++) {
+            const size_t ra = (size_t)R.uniq[c.u] * H + 16 * (rb0 + c.rbl) + g;
+            const uint8_t *cp = W.down_codes + ra * (I / 2) + 64 * c.r + 16 * q;
+            const uint8_t *sp = W.down_scales + ra * (I / 16) + 8 * c.r + 2 * q;
+            b.ca[j] = ldg_stream(cp);
+            b.cb[j] = ldg_stream(cp + 8 * (I / 2));
+            b.sa[j] = __ldg(reinterpret_cast<const unsigned short *>(sp));
+            b.sb[j] = __ldg(reinterpret_cast<const unsigned short *>(sp + 8 * (I / 16)));
+            if (j + 1 < n) dn_next(c, U, R2);
+        }
+        return;
+    }
 #pragma unroll
     for (int j = 0; j < kDnUnits; j++) {
         if (j < n) {
@@ -373,11 +403,11 @@ __device__ inline void dn_issue(const Params &p, const DecLayer &W, const DecRou
                 const uint8_t *sp = W.down_scales + ra * (I / 16) + 8 * c.r + 2 * q;
                 b.ca[j] = ldg_stream(cp);
                 b.cb[j] = ldg_stream(cp + 8 * (I / 2));
-                b.s[j] = (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sp)) |
-                         ((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(sp + 8 * (I / 16))) << 16);
+                b.sa[j] = __ldg(reinterpret_cast<const unsigned short *>(sp));
+                b.sb[j] = __ldg(reinterpret_cast<const unsigned short *>(sp + 8 * (I / 16)));
             } else {
                 b.ca[j] = b.cb[j] = make_uint4(0, 0, 0, 0);
-                b.s[j] = 0;
+                b.sa[j] = b.sb[j] = 0;
             }
             dn_next(c, U, R2);
         }
@@ -541,6 +571,7 @@ __device__ __forceinline__ void decode_body(const Params &p, const DecLayer &W, 
     // are staged
     const int R1 = cdiv(H, 128), R2 = cdiv(I, 128);
     const bool gvec = H % 128 == 0 && ((uintptr_t)W.gate_scales | (uintptr_t)W.up_scales) % 8 == 0;
+    const bool dfull = I % 128 == 0;
     const int n1 = (ge - gb) * R1;
     int a1, b1;
     share(n1, warp, kDecWarps, a1, b1);
@@ -607,7 +638,7 @@ __device__ __forceinline__ void decode_body(const Params &p, const DecLayer &W, 
     int a2, b2;
     share(n2, warp, kDecWarps, a2, b2);
     DnBuf d0, d1;
-    dn_issue(p, W, R, rb0, dn_cur(a2, U, R2), min(kDnUnits, b2 - a2), g, q, d0);
+    dn_issue(p, W, R, rb0, dn_cur(a2, U, R2), min(kDnUnits, b2 - a2), g, q, dfull, d0);
     __syncthreads();
     // granules split between warps: their parts summed in warp order
     for (int j = warp; j < ge - gb; j += kDecWarps) {
@@ -668,7 +699,7 @@ __device__ __forceinline__ void decode_body(const Params &p, const DecLayer &W, 
                 DnCur ic = cc;   // the next chunk starts kDnUnits units on
 #pragma unroll
                 for (int j = 0; j < kDnUnits; j++) dn_next(ic, U, R2);
-                dn_issue(p, W, R, rb0, ic, min(kDnUnits, b2 - xn), g, q, nb);
+                dn_issue(p, W, R, rb0, ic, min(kDnUnits, b2 - xn), g, q, dfull, nb);
             }
 #pragma unroll
             for (int j = 0; j < kDnUnits; j++) {
@@ -678,7 +709,7 @@ __device__ __forceinline__ void decode_body(const Params &p, const DecLayer &W, 
                     dn_next(cc, U, R2);
                     const int pos = g < T ? R.upos[u * kSlots + g] : -1;
                     const __half *hr = hs + (size_t)(pos >= 0 ? pos : T * p.K) * ld2 + 128 * r + 32 * q;
-                    round_mma(acc, b.ca[j], b.cb[j], b.s[j] & 0xFFFF, b.s[j] >> 16,
+                    round_mma(acc, b.ca[j], b.cb[j], b.sa[j], b.sb[j],
                               [&](int s, uint32_t &v0, uint32_t &v1) {
                                   const uint2 v = *reinterpret_cast<const uint2 *>(hr + 4 * s);
                                   v0 = v.x;

@@ -79,9 +79,18 @@ struct SeBuf {
 // row's end are zero, with zero scales.
 template <int NR>
 __device__ inline void se_issue(int c, const uint8_t *ac, const uint8_t *bc, const uint8_t *as,
-                                const uint8_t *bs, int kb, bool v32, bool vec, int q, SeBuf<NR> &b) {
+                                const uint8_t *bs, int kb, bool v32, bool vec, bool full, int q, SeBuf<NR> &b) {
     const int c0 = 64 * NR * c + 16 * NR * q;   // first code byte of this quarter
     const int s0 = 8 * NR * c + 2 * NR * q;     // first scale byte
+    if (NR == 2 && full) {
+        // every chunk whole, 32-byte code and 4-byte scale loads allowed: all loads
+        // unconditional, each landing straight in its buffer register
+        ldg_stream32(ac + c0, b.ca[0], b.ca[NR - 1]);
+        ldg_stream32(bc + c0, b.cb[0], b.cb[NR - 1]);
+        b.sa[0] = __ldg(reinterpret_cast<const uint32_t *>(as + s0));
+        b.sb[0] = __ldg(reinterpret_cast<const uint32_t *>(bs + s0));
+        return;
+    }
     if (c0 + 16 * NR <= kb) {
         if (NR == 2 && v32) {
             ldg_stream32(ac + c0, b.ca[0], b.ca[NR - 1]);
@@ -224,6 +233,7 @@ __global__ void __launch_bounds__(kSeThreads, 1) small_expert_kernel(Params p) {
     const uint8_t *cbase_a = MODE == 0 ? p.gate_codes : p.down_codes;
     const uint8_t *cbase_b = MODE == 0 ? p.up_codes : p.down_codes;
     const bool v32 = kb % 32 == 0 && ((uintptr_t)cbase_a | (uintptr_t)cbase_b) % 32 == 0;
+    const bool full = v32 && vec && Kin % (128 * NR) == 0;
     const int S = se_pieces(nse, units, gridDim.x);
     if (nse > 0) {
         uint4 *z = reinterpret_cast<uint4 *>(se_sm);
@@ -259,7 +269,7 @@ __global__ void __launch_bounds__(kSeThreads, 1) small_expert_kernel(Params p) {
         // issues the chunk at the issue cursor into b and advances the cursor
         auto issue = [&](SeBuf<NR> &b) {
             const int ra = rstep * igr + g, rb = ra + roff_b;
-            se_issue<NR>(ic, ca_e + ra * kb, cb_e + rb * kb, sa_e + ra * ks, sb_e + rb * ks, kb, v32, vec, q, b);
+            se_issue<NR>(ic, ca_e + ra * kb, cb_e + rb * kb, sa_e + ra * ks, sb_e + rb * ks, kb, v32, vec, full, q, b);
             if (++ic == C) {
                 ic = 0;
                 igr++;
