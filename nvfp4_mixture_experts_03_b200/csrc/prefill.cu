@@ -64,8 +64,8 @@ constexpr uint64_t kSettleNs = 1000000ull;     // lets in-flight copies land aft
 constexpr uint16_t kBothCtas = 0x3;
 
 struct __align__(8) Bars {
-    uint64_t a_full[kRing];     // leader: 8 dequant warps x 2 CTAs
-    uint64_t b_full[kRing];     // leader: expect_tx of both halves
+    uint64_t a_full[kRing];     // leader: 8 dequant warps x 2 CTAs, and the B warp's expect_tx
+                                //   for both halves of B (one barrier per stage for the MMA)
     uint64_t empty[kRing];      // both: the pair MMA's commit
     uint64_t raw_full[kRawStages];   // code bytes (TMA) + 32 scale-copy lanes
     uint64_t raw_empty[kRawStages];  // 8 dequant warps
@@ -107,6 +107,18 @@ struct Ring {
 // First weight row of this CTA's 128-row half of tile t (down: the second half of
 // the last tile lies past H when H % 256 == 128; it then reads the first half's
 // rows, in bounds, and its results are dropped).
+// Non-blocking test: has the phase with this parity completed?
+__device__ inline bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 template <int MODE>
 __device__ inline int half_row0(const Params &p, const Tile &t, int rank) {
     if (MODE == 0) return t.expert * p.I + t.m0 + kGuCta * rank;
@@ -235,8 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRing; s++) {
-            mbar_init(&bars->a_full[s], 16);
-            mbar_init(&bars->b_full[s], 1);
+            mbar_init(&bars->a_full[s], 17);
             mbar_init(&bars->empty[s], 1);
         }
         for (int b = 0; b < 2; b++) {
@@ -402,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 12) {
         // ------------------------------------------------------ TMA for B
         // This CTA's half of the tile's pair rows, in 64-row boxes; the bytes are
-        // counted on the leader's b_full, whose single arrival (with the byte
+        // counted on the leader's a_full, whose one arrival from this warp (with the byte
         // count of both halves) the leader makes. The next tile's descriptor is
         // read one tile ahead.
         if (lane == 0) {
@@ -423,11 +434,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nbox = cdiv(half, kBBox);
                 uint8_t *bs = b_base + ring.stage * kBStage;
                 if (leader) {
-                    mbar_arrive_expect_tx(&bars->b_full[ring.stage], 2 * nbox * kBoxBytes);
+                    mbar_arrive_expect_tx(&bars->a_full[ring.stage], 2 * nbox * kBoxBytes);
                     issued |= 1u << ring.stage;
                     issued_phase = (issued_phase & ~(1u << ring.stage)) | (ring.phase << ring.stage);
                 }
-                const uint32_t bar = mapa_shared(&bars->b_full[ring.stage], 0);
+                const uint32_t bar = mapa_shared(&bars->a_full[ring.stage], 0);
                 for (int b = 0; b < nbox; b++)
                     tma_load_2d_pair(bs + b * kBoxBytes, &map_b, bar, cs.kk * kBK,
                                      t.pos0 + rank * half + b * kBBox);
@@ -437,14 +448,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             // The leader's last load of every stage must have landed before exit.
             for (int s = 0; s < kRing; s++)
                 if (issued & (1u << s))
-                    mbar_wait_drain(&bars->b_full[s], (issued_phase >> s) & 1, kDrainNs);
+                    mbar_wait_drain(&bars->a_full[s], (issued_phase >> s) & 1, kDrainNs);
         }
     } else if (warp == 13) {
         // ---------------------------------------------- pair MMA issue (leader)
         if (leader && lane == 0) {
+            // This one thread paces the tile: per K step it used to spend about as
+            // long waiting on two already-complete barriers and computing
+            // descriptors as issuing the four MMAs. So: one barrier per stage
+            // (A arrivals and B bytes together), the next stage's barrier tested
+            // without blocking while this stage's MMAs go out, and each stage's
+            // descriptors computed once (the k16 steps add 32 bytes, i.e. 2, to
+            // the address field).
             Ring<kRing> ring;
             uint32_t acc_phase = 0;     // bit b: parity of accumulator b's next use
             bool ok = true;
+            uint64_t adesc[kRing], bdesc[kRing];
+#pragma unroll
+            for (int st = 0; st < kRing; st++) {
+                adesc[st] = smem_desc_sw128(smem_u32(a_base + st * kAStage));
+                bdesc[st] = smem_desc_sw128(smem_u32(b_base + st * kBStage));
+            }
+            bool ready = false;   // the current stage's barrier already seen complete
             for (int tl = 0; ok && tl < ntl; tl++) {
                 const Tile t = tiles[cid + tl * ncl];
                 const int buf = tl & 1;
@@ -455,21 +480,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc_phase ^= 1u << buf;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * kBN;
-                for (int kk = 0; kk < nk; kk++) {
-                    if (!mbar_wait(&bars->a_full[ring.stage], ring.phase, abort, p.status, 5) ||
-                        !mbar_wait(&bars->b_full[ring.stage], ring.phase, abort, p.status, 6)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t as = smem_u32(a_base + ring.stage * kAStage);
-                    const uint32_t bs = smem_u32(b_base + ring.stage * kBStage);
+                // two K steps per iteration (nk is even)
+                for (int kk = 0; kk < nk; kk += 2) {
 #pragma unroll
-                    for (int k16 = 0; k16 < kBK / 16; k16++)
-                        tc_mma_f16_pair(d_tmem, smem_desc_sw128(as + 32 * k16),
-                                        smem_desc_sw128(bs + 32 * k16), idesc, (kk | k16) != 0);
-                    tc_commit_pair_mc(&bars->empty[ring.stage], kBothCtas);
-                    ring.next();
+                    for (int h2 = 0; h2 < 2; h2++) {
+                        if (!ready && !mbar_wait(&bars->a_full[ring.stage], ring.phase, abort, p.status, 5)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        Ring<kRing> nx = ring;
+                        nx.next();
+                        ready = mbar_test(&bars->a_full[nx.stage], nx.phase);
+                        uint64_t ad = adesc[0], bd = bdesc[0];
+#pragma unroll
+                        for (int st = 1; st < kRing; st++)
+                            if (ring.stage == st) {
+                                ad = adesc[st];
+                                bd = bdesc[st];
+                            }
+#pragma unroll
+                        for (int k16 = 0; k16 < kBK / 16; k16++)
+                            tc_mma_f16_pair(d_tmem, ad + 2 * k16, bd + 2 * k16, idesc, ((kk + h2) | k16) != 0);
+                        tc_commit_pair_mc(&bars->empty[ring.stage], kBothCtas);
+                        ring = nx;
+                    }
+                    if (!ok) break;
                 }
                 if (ok) tc_commit_pair_mc(&bars->acc_full[buf], kBothCtas);
             }
