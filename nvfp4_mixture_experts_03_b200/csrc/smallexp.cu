@@ -5,9 +5,9 @@
 // ("Strata NVFP4" README, "How it differs from upstream Strata"); their
 // MoE layers route by top-k over many experts, so a skewed batch leaves a long
 // tail of experts with a handful of tokens. A tensor-core tile of the grouped
-// GEMM costs nearly the same for 4 tokens as for 256 (its K loop is bound by
-// the weight stream and the E2M1 conversion), so those experts are taken out of
-// the tile lists and streamed here instead, like the decode layer does: each
+// GEMM costs nearly the same for 4 tokens as for 256 (the time of a K step
+// hardly depends on the tile's N), so those experts are taken out of the tile
+// lists and streamed here instead, like the decode layer does: each
 // weight byte is read once into registers, decoded exactly to F16 and fed to
 // mma.sync m16n8k16 with the expert's pairs as N (two 8-pair halves sharing
 // each decoded weight fragment), FP32 accumulation.
