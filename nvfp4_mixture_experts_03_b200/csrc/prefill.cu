@@ -453,13 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 13) {
         // ---------------------------------------------- pair MMA issue (leader)
         if (leader && lane == 0) {
-            // This one thread paces the tile: per K step it used to spend about as
-            // long waiting on two already-complete barriers and computing
-            // descriptors as issuing the four MMAs. So: one barrier per stage
-            // (A arrivals and B bytes together), the next stage's barrier tested
-            // without blocking while this stage's MMAs go out, and each stage's
-            // descriptors computed once (the k16 steps add 32 bytes, i.e. 2, to
-            // the address field).
+            // This one thread paces the tile (the operands are almost always ready
+            // when it gets to them), so its K step is kept short: one barrier per
+            // stage (A arrivals and B bytes together), the next stage's barrier
+            // tested without blocking while this stage's MMAs go out, each stage's
+            // descriptors computed once (a k16 step adds 32 bytes, i.e. 2, to the
+            // address field), two K steps per loop iteration.
             Ring<kRing> ring;
             uint32_t acc_phase = 0;     // bit b: parity of accumulator b's next use
             bool ok = true;
