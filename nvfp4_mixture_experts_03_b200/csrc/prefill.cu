@@ -45,17 +45,19 @@ constexpr int kThreads = 480;
 constexpr int kBM = 128;                       // A rows per CTA (the pair MMA has M = 256)
 constexpr int kGuCta = kGuRows / 2;            // intermediates per CTA in a gate/up tile
 constexpr int kBRows = kBN / 2;                // B rows per CTA
-constexpr int kAStage = kBM * kBK * 2;         // 16 KB
-constexpr int kBStage = kBRows * kBK * 2;      // 16 KB
+constexpr int kSub = 2;                        // 64-wide K blocks (one 128-byte swizzle row each) per stage
+constexpr int kSubBytes = kBM * kBK * 2;       // 16 KB: one block of A (or of B) per CTA
+constexpr int kAStage = kSub * kSubBytes;      // 32 KB: 128 K of A
+constexpr int kBStage = kSub * kBRows * kBK * 2;   // 32 KB: 128 K of B
 constexpr int kBBox = 64;                      // rows per TMA box
 constexpr int kBoxBytes = kBBox * kBK * 2;     // 8 KB
-constexpr int kRing = 4;                       // A/B pipeline stages
+constexpr int kRing = 2;                       // A/B pipeline stages of 128 K (eight MMAs each)
 constexpr int kRawSteps = 4;                   // K steps per raw weight stage
 constexpr int kRawStages = 4;                  // 16 K steps of weights in flight: covers HBM latency
 constexpr int kRawCodeBytes = kBM * kRawSteps * 32;   // 128 rows x 128 B of E2M1 codes
 constexpr int kRawScaleBytes = kBM * kRawSteps * 4;   // 128 rows x 16 B of E4M3 scales
 constexpr int kRawBytes = kRawCodeBytes + kRawScaleBytes;
-static_assert(kRing % 2 == 0 && kRawSteps % 2 == 0, "the dequant warps fill ring stages in pairs");
+static_assert(kRawSteps % kSub == 0 && kBRows * kBK * 2 == kSubBytes, "a raw stage holds whole ring stages");
 constexpr int kTmemCols = 512;                 // two 256-column accumulators
 constexpr int kEpiBytes = 2 * 32 * kBM * 2;    // epilogue staging: 2 x (32 columns x 128 rows x F16)
 constexpr int kColBytes = kBN * 4;            // one per-column factor array of a tile (FP32)
@@ -288,9 +290,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         Ring<kRawStages> rr;
         uint4 s4 = make_uint4(0, 0, 0, 0);
         bool ok = true;
-        // Two K steps (two ring stages) per iteration: K is a multiple of 128, so
-        // every tile has an even number of steps and the pair never wraps the ring
-        // (kRing is even); one proxy fence and one pass of waits per pair.
+        // One ring stage (two 64-wide K blocks) per iteration: K is a multiple of
+        // 128, so every tile has an even number of 64-wide steps; one wait, one
+        // proxy fence and one arrival per stage.
         for (int tl = 0; ok && tl < ntl; tl++) {
             for (int kk = 0; kk < nk; kk += 2) {
                 const int kq = kk % kRawSteps;   // 0 or 2
@@ -303,9 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     s4 = *reinterpret_cast<const uint4 *>(raw + scale_off);
                 }
-                const int s0 = ring.stage, s1 = ring.stage + 1;
-                const bool got = mbar_wait(&bars->empty[s0], ring.phase ^ 1, abort, p.status, 1) &&
-                                 mbar_wait(&bars->empty[s1], ring.phase ^ 1, abort, p.status, 1);
+                const int s0 = ring.stage;
+                const bool got = mbar_wait(&bars->empty[s0], ring.phase ^ 1, abort, p.status, 1);
                 if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
                     break;
@@ -314,14 +315,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint4 code1 = *reinterpret_cast<const uint4 *>(raw + code_off + (((2 * kq + 2 + hf) ^ swz) << 4));
                 const uint32_t sw0 = kq == 0 ? s4.x : s4.z, sw1 = kq == 0 ? s4.y : s4.w;
                 store_half_row(a_base + s0 * kAStage, r, hf, code0, sw0 >> (16 * hf));
-                store_half_row(a_base + s1 * kAStage, r, hf, code1, sw1 >> (16 * hf));
+                store_half_row(a_base + s0 * kAStage + kSubBytes, r, hf, code1, sw1 >> (16 * hf));
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive_cluster(mapa_shared(&bars->a_full[s0], 0));
-                    mbar_arrive_cluster(mapa_shared(&bars->a_full[s1], 0));
-                }
-                ring.next();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(&bars->a_full[s0], 0));
                 ring.next();
                 if (kq + 1 == kRawSteps - 1 || kk + 2 == nk) {
                     __syncwarp();
@@ -417,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // count of both halves) the leader makes. The next tile's descriptor is
         // read one tile ahead.
         if (lane == 0) {
-            Cursor cs(nk, ntiles, cid, ncl);
+            Cursor cs(nk / kSub, ntiles, cid, ncl);   // steps over ring stages (128 K)
             Ring<kRing> ring;
             uint32_t issued = 0, issued_phase = 0;  // leader: stages with a load in flight
             int cur_tile = -1;
@@ -434,14 +431,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nbox = cdiv(half, kBBox);
                 uint8_t *bs = b_base + ring.stage * kBStage;
                 if (leader) {
-                    mbar_arrive_expect_tx(&bars->a_full[ring.stage], 2 * nbox * kBoxBytes);
+                    mbar_arrive_expect_tx(&bars->a_full[ring.stage], kSub * 2 * nbox * kBoxBytes);
                     issued |= 1u << ring.stage;
                     issued_phase = (issued_phase & ~(1u << ring.stage)) | (ring.phase << ring.stage);
                 }
                 const uint32_t bar = mapa_shared(&bars->a_full[ring.stage], 0);
-                for (int b = 0; b < nbox; b++)
-                    tma_load_2d_pair(bs + b * kBoxBytes, &map_b, bar, cs.kk * kBK,
-                                     t.pos0 + rank * half + b * kBBox);
+                for (int sb = 0; sb < kSub; sb++)
+                    for (int b = 0; b < nbox; b++)
+                        tma_load_2d_pair(bs + sb * kSubBytes + b * kBoxBytes, &map_b, bar,
+                                         (kSub * cs.kk + sb) * kBK, t.pos0 + rank * half + b * kBBox);
                 ring.next();
                 cs.next();
             }
@@ -458,7 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // stage (A arrivals and B bytes together), the next stage's barrier
             // tested without blocking while this stage's MMAs go out, each stage's
             // descriptors computed once (a k16 step adds 32 bytes, i.e. 2, to the
-            // address field), two K steps per loop iteration.
+            // address field; the second 64-wide block of a stage 16 KB), and
+            // stages of 128 K: eight MMAs per wait, test and commit.
             Ring<kRing> ring;
             uint32_t acc_phase = 0;     // bit b: parity of accumulator b's next use
             bool ok = true;
@@ -479,32 +478,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc_phase ^= 1u << buf;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * kBN;
-                // two K steps per iteration (nk is even)
-                for (int kk = 0; kk < nk; kk += 2) {
+                // one ring stage (two 64-wide K blocks, eight MMAs) per iteration
+                for (int ks = 0; ks < nk / kSub; ks++) {
+                    if (!ready && !mbar_wait(&bars->a_full[ring.stage], ring.phase, abort, p.status, 5)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    Ring<kRing> nx = ring;
+                    nx.next();
+                    ready = mbar_test(&bars->a_full[nx.stage], nx.phase);
+                    uint64_t ad = adesc[0], bd = bdesc[0];
 #pragma unroll
-                    for (int h2 = 0; h2 < 2; h2++) {
-                        if (!ready && !mbar_wait(&bars->a_full[ring.stage], ring.phase, abort, p.status, 5)) {
-                            ok = false;
-                            break;
+                    for (int st = 1; st < kRing; st++)
+                        if (ring.stage == st) {
+                            ad = adesc[st];
+                            bd = bdesc[st];
                         }
-                        tc_fence_after();
-                        Ring<kRing> nx = ring;
-                        nx.next();
-                        ready = mbar_test(&bars->a_full[nx.stage], nx.phase);
-                        uint64_t ad = adesc[0], bd = bdesc[0];
 #pragma unroll
-                        for (int st = 1; st < kRing; st++)
-                            if (ring.stage == st) {
-                                ad = adesc[st];
-                                bd = bdesc[st];
-                            }
+                    for (int sb = 0; sb < kSub; sb++)
 #pragma unroll
                         for (int k16 = 0; k16 < kBK / 16; k16++)
-                            tc_mma_f16_pair(d_tmem, ad + 2 * k16, bd + 2 * k16, idesc, ((kk + h2) | k16) != 0);
-                        tc_commit_pair_mc(&bars->empty[ring.stage], kBothCtas);
-                        ring = nx;
-                    }
-                    if (!ok) break;
+                            tc_mma_f16_pair(d_tmem, ad + sb * (kSubBytes >> 4) + 2 * k16,
+                                            bd + sb * (kSubBytes >> 4) + 2 * k16, idesc, (ks | sb | k16) != 0);
+                    tc_commit_pair_mc(&bars->empty[ring.stage], kBothCtas);
+                    ring = nx;
                 }
                 if (ok) tc_commit_pair_mc(&bars->acc_full[buf], kBothCtas);
             }
