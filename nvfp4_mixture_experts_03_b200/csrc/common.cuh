@@ -435,8 +435,11 @@ struct CodeMaps {
     CUtensorMap gate, up, down;
 };
 // Clusters of two CTAs, at most `max_clusters` of them (persistent).
+// map_y: the per-pair down rows (xh) as a bulk-store target, boxes of 32 pairs x
+// 128 hidden rows (used by mode 1)
 cudaError_t launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &map_b,
-                                const CodeMaps &codes, int max_clusters, cudaStream_t s);
+                                const CodeMaps &codes, const CUtensorMap &map_y, int max_clusters,
+                                cudaStream_t s);
 // Per device: opt the GEMM kernels into their shared memory; *max_clusters = how
 // many CTA pairs of either GEMM can be resident at once.
 cudaError_t prefill_init(int *max_clusters);

@@ -69,6 +69,21 @@ bool make_map_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// F16 [rows][cols] as a bulk-store target: unswizzled boxes of box_cols x
+// box_rows, laid out in shared memory row after row.
+bool make_map_f16_store(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_cols,
+                        int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Packed E2M1 code plane [rows][cols] bytes: 128-byte x box_rows boxes, swizzled
 // like the GEMM's shared-memory tiles.
 bool make_map_codes(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows) {
@@ -377,8 +392,9 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
         mark(4);
     } else {
         const int64_t P = (int64_t)T * d.top_k;
-        CUtensorMap map_xh, map_h;
-        if (!make_map_f16(&map_xh, p.xh, P, d.hidden, 64) || !make_map_f16(&map_h, p.h, P, d.inter, 64))
+        CUtensorMap map_xh, map_h, map_y;
+        if (!make_map_f16(&map_xh, p.xh, P, d.hidden, 64) || !make_map_f16(&map_h, p.h, P, d.inter, 64) ||
+            !make_map_f16_store(&map_y, p.xh, P, d.hidden, 128, 32))
             return NVFP4_MOE_ERR_CUDA;
         mark(0);
         if (router && launch_router(p, s) != cudaSuccess) return NVFP4_MOE_ERR_CUDA;
@@ -386,11 +402,11 @@ int nvfp4_moe_forward(nvfp4_moe_t *h, const nvfp4_moe_io *io, void *ws, size_t w
         mark(1);
         launch_prep_prefill(p, s);
         mark(2);
-        if (launch_prefill_gemm(0, p, map_xh, h->codes, h->pf_clusters, s) != cudaSuccess ||
+        if (launch_prefill_gemm(0, p, map_xh, h->codes, map_y, h->pf_clusters, s) != cudaSuccess ||
             launch_small(0, p, s) != cudaSuccess)
             return NVFP4_MOE_ERR_CUDA;
         mark(3);
-        if (launch_prefill_gemm(1, p, map_h, h->codes, h->pf_clusters, s) != cudaSuccess ||
+        if (launch_prefill_gemm(1, p, map_h, h->codes, map_y, h->pf_clusters, s) != cudaSuccess ||
             launch_small(1, p, s) != cudaSuccess)
             return NVFP4_MOE_ERR_CUDA;
         launch_combine(p, s);

@@ -109,6 +109,19 @@ struct Ring {
 // First weight row of this CTA's 128-row half of tile t (down: the second half of
 // the last tile lies past H when H % 256 == 128; it then reads the first half's
 // rows, in bounds, and its results are dropped).
+// Bulk tensor store of a shared-memory box (no swizzle) to global, in this
+// thread's bulk group; commit and waits for the groups this thread issued.
+__device__ inline void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ inline void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// all but the newest group have finished reading their shared memory
+__device__ inline void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// every group has completed (its global writes done)
+__device__ inline void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Non-blocking test: has the phase with this parity completed?
 __device__ inline bool mbar_test(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
@@ -218,7 +231,8 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const Params p, const __grid_constant__ CUtensorMap map_b,
                         const __grid_constant__ CUtensorMap map_a0,
-                        const __grid_constant__ CUtensorMap map_a1) {
+                        const __grid_constant__ CUtensorMap map_a1,
+                        const __grid_constant__ CUtensorMap map_y) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
@@ -613,6 +627,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < kChunks; c++) {
                         if (32 * c >= t.ntok) break;
                         __half *ys = reinterpret_cast<__half *>(epi_stage) + (c & 1) * (32 * kBM);
+                        // A whole chunk (32 pairs, 128 rows inside H) leaves by one bulk
+                        // tensor store from this staging buffer; the store issued from it
+                        // two chunks ago must have finished reading it first.
+                        const bool whole = t.ntok - 32 * c >= 32 && nr == kBM;
+                        if (threadIdx.x == 0) bulk_wait_read_1();
+                        epi_sync();
                         // The chunk's 32 column factors in registers before the first
                         // staging store.
                         float cf[32];
@@ -631,9 +651,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                             fin &= fits_f16(yf) || !row_ok;
                             ys[j * kBM + r] = __float2half_rn(yf);
                         }
-                        epi_sync();
-                        store_chunk<kBM>(ys, p.xh + (size_t)(t.pos0 + 32 * c) * p.H + m, p.H,
-                                         min(32, t.ntok - 32 * c), nr);
+                        if (whole) {
+                            fence_proxy_async_smem();   // the staging writes, before the bulk copy reads them
+                            epi_sync();
+                            if (threadIdx.x == 0) {
+                                tma_store_2d(&map_y, ys, m, t.pos0 + 32 * c);
+                                bulk_commit();
+                            }
+                        } else {
+                            epi_sync();
+                            store_chunk<kBM>(ys, p.xh + (size_t)(t.pos0 + 32 * c) * p.H + m, p.H,
+                                             min(32, t.ntok - 32 * c), nr);
+                        }
                     }
                 }
                 // the per-pair rows w * s_d * y are stored in F16 (see above)
@@ -643,6 +672,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(&bars->acc_empty[buf], 0));
         }
+        // every bulk store of the down rows complete before the CTA ends
+        if (threadIdx.x == 0) bulk_wait_all();
     }
 
     __syncwarp();
@@ -695,12 +726,13 @@ cudaError_t prefill_init(int *max_clusters) {
 }
 
 cudaError_t launch_prefill_gemm(int mode, const Params &p, const CUtensorMap &map_b,
-                                const CodeMaps &codes, int max_clusters, cudaStream_t s) {
+                                const CodeMaps &codes, const CUtensorMap &map_y, int max_clusters,
+                                cudaStream_t s) {
     const int maxt = mode == 0 ? p.max_tiles_gu : p.max_tiles_dn;
     cudaLaunchAttribute attr[1];
     const cudaLaunchConfig_t cfg = gemm_config(max(1, min(max_clusters, maxt)), s, attr);
-    return mode == 0 ? cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<0>, p, map_b, codes.gate, codes.up)
-                     : cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<1>, p, map_b, codes.down, codes.down);
+    return mode == 0 ? cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<0>, p, map_b, codes.gate, codes.up, map_y)
+                     : cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<1>, p, map_b, codes.down, codes.down, map_y);
 }
 
 }  // namespace nvmoe
