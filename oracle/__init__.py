@@ -192,6 +192,41 @@ def decode_matrix(codes, scales, glob) -> np.ndarray:
     return out
 
 
+def quantize_act_nvfp4(x_bf16):
+    """Activations as an FP4 x FP4 prompt path multiplies them ("Strata NVFP4"
+    README, "How it differs from upstream Strata", the W4A8 bullet: llama.cpp's
+    NVFP4 prompt path on sm_120 runs FP4 x FP4). The pages do not print the
+    activation recipe; the reading taken is the checkpoint's own NVFP4 recipe
+    applied per token: each token row is one tensor for `quantize` (global =
+    amax / (6 * 448) in FP32, an E4M3 scale per 16 elements, E2M1 codes nearest).
+    x: BF16 [T][H] (torch bf16 or uint16 bits) ->
+    (codes u8 [T][H/2], scales u8 [T][H/16], glob f32 [T])."""
+    x = _np(x_bf16).view(np.uint16)
+    codes, scales, glob = quantize(np.ascontiguousarray(x[:, None, :]))
+    return codes[:, 0], scales[:, 0], glob
+
+
+def dequant_act_nvfp4(codes, scales, glob) -> np.ndarray:
+    """FP64 [T][H] values of per-token NVFP4 activations (each row decoded with
+    its own global)."""
+    return np.concatenate([decode_matrix(codes[t:t + 1], scales[t:t + 1], glob[t])
+                           for t in range(len(glob))])
+
+
+def quantize_act_int8(x_bf16):
+    """Per-token symmetric int8, the activation format of the W4A8 prompt path
+    ("Strata NVFP4" README, "How it differs from upstream Strata", the W4A8 bullet:
+    8-bit activations), as this layer takes it: scale_t = amax_t / 127 rounded to
+    FP32, q = nearest integer of x / scale_t (ties to even), clamped to +-127.
+    -> (q int8 [T][H], scale f32 [T])."""
+    x = _np(x_bf16).view(np.uint16)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    scale = (np.abs(xf).max(axis=1) / 127.0).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float64)
+    q = np.clip(np.rint(xf / safe[:, None]), -127, 127).astype(np.int8)
+    return q, scale
+
+
 class _Bound:
     """ctypes views of one layer's planes (keeps the numpy arrays alive)."""
 

@@ -158,6 +158,72 @@ def test_quantiser_round_trip_and_error_bound():
     assert np.all(same)
 
 
+# ------------------------------------------- activation formats (FP4 x FP4 study)
+
+_E2M1_VALS = np.array([v for m in brute.E2M1_MAGNITUDES for v in (m, -m)])
+
+
+def test_nvfp4_activations_exact_values_round_trip():
+    # rows built from exact NVFP4 values: each block holds a +-6 code so that its
+    # amax is 6 x its E4M3 scale x a power-of-two global, and one block per row
+    # sits at scale 448 so that the global is amax / (6 * 448) exactly
+    g = torch.Generator().manual_seed(11)
+    T, H = 3, 64
+    mags = torch.tensor(brute.E2M1_MAGNITUDES, dtype=torch.float64)
+    e4 = torch.arange(1, 127, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+    e4 = e4.to(torch.float64)
+    x = torch.zeros(T, H, dtype=torch.float64)
+    for t in range(T):
+        glob = 2.0 ** (-12 + 3 * t)
+        for b in range(H // 16):
+            sc = 448.0 if b == t % (H // 16) else float(e4[torch.randint(0, len(e4), (1,), generator=g)])
+            v = mags[torch.randint(0, 8, (16,), generator=g)]
+            v = v * torch.where(torch.rand(16, generator=g) < 0.5, -1.0, 1.0)
+            v[int(torch.randint(0, 16, (1,), generator=g))] = 6.0
+            x[t, 16 * b:16 * b + 16] = v * sc * glob
+    xb = x.to(torch.bfloat16)
+    assert torch.equal(xb.to(torch.float64), x)          # exact in BF16
+    c, s, gl = oracle.quantize_act_nvfp4(xb)
+    assert np.array_equal(oracle.dequant_act_nvfp4(c, s, gl), x.numpy())
+    assert np.array_equal(gl.astype(np.float64), [2.0 ** (-12 + 3 * t) for t in range(T)])
+
+
+def test_nvfp4_activations_pick_the_nearest_block_scale_and_code():
+    x = synth.make_x_bf16(5, 128, seed=12, outliers=True)
+    c, s, gl = oracle.quantize_act_nvfp4(x)
+    xf = x.to(torch.float64).numpy()
+    e4 = torch.arange(0, 127, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+    e4 = e4.to(torch.float64).numpy()
+    for t in range(5):
+        assert gl[t] == np.float32(np.abs(xf[t]).max() / (6.0 * 448.0))
+        g = float(gl[t])
+        for b in range(128 // 16):
+            blk = xf[t, 16 * b:16 * b + 16]
+            want = np.abs(blk).max() / g / 6.0
+            sb = int(s[t, b])
+            assert abs(e4[sb] - want) <= np.abs(e4 - want).min()   # nearest E4M3 scale
+            step = e4[sb] * g
+            q = brute.dense(c[t:t + 1, 8 * b:8 * b + 8], s[t:t + 1, b:b + 1], g)[0]
+            for k in range(16):                                     # nearest code at that scale
+                assert abs(q[k] - blk[k]) <= np.abs(_E2M1_VALS * step - blk[k]).min() * (1 + 1e-12)
+
+
+def test_int8_activations_round_trip_and_half_step_bound():
+    q0 = torch.randint(-127, 128, (4, 96), generator=torch.Generator().manual_seed(13))
+    q0[:, 5] = 127
+    sc = torch.tensor([2.0 ** -7, 2.0 ** -3, 0.5, 4.0], dtype=torch.float64)
+    x = (q0.to(torch.float64) * sc[:, None]).to(torch.bfloat16)
+    assert torch.equal(x.to(torch.float64), q0.to(torch.float64) * sc[:, None])
+    q, s = oracle.quantize_act_int8(x)
+    assert np.array_equal(q.astype(np.int64), q0.numpy()) and np.array_equal(s, sc.numpy())
+    y = synth.make_x_bf16(6, 200, seed=14, outliers=True)
+    q, s = oracle.quantize_act_int8(y)
+    yf = y.to(torch.float64).numpy()
+    err = np.abs(q.astype(np.float64) * s[:, None].astype(np.float64) - yf)
+    assert np.all(err <= 0.5 * s[:, None].astype(np.float64) * (1 + 1e-6))
+    assert np.all(np.abs(q).max(axis=1) == 127)
+
+
 # ----------------------------------------------------------------- routing
 
 def test_route_matches_library_sort_and_softmax():
