@@ -8,7 +8,8 @@
 // ("strata-5090-4070" README, "RAM: the one thing to know"), which is why a tile
 // covers up to 256 pairs of one expert.
 //
-// Operands, per 64-wide K stage, in each CTA of the pair:
+// Operands, per ring stage of 128 K (two 64-wide K blocks), in each CTA of the
+// pair:
 //   A (weights, 128 of the tile's 256 rows): dequantised by eight warps from the
 //     packed planes straight into the 128-byte-swizzled K-major layout. code x
 //     E4M3 scale is exact in F16, so the MMA sees the stored weights without
@@ -26,11 +27,12 @@
 // Epilogues: gate/up -> scales, SwiGLU, F16 h at the pair's position (each CTA
 // owns 64 intermediates: 64 gate rows and the 64 matching up rows, arranged so
 // that each TMEM lane quarter holds 16 gate and the matching 16 up rows);
-// down -> scale x routing weight, F16 row per pair (combined per token by a
-// separate deterministic kernel).
+// down -> scale x routing weight, F16 row per pair (whole 32-pair chunks leave
+// by one bulk tensor store; combined per token by a separate deterministic
+// kernel).
 //
-// Warp roles (480 threads per CTA): 0-3 epilogue, 4-11 dequantise A (two warps
-// per row: one for each half of the 64-wide K stage), 12 TMA for B, 13 TMEM
+// Warp roles (480 threads per CTA): 0-3 epilogue, 4-11 dequantise A (two threads
+// per row: one for each half of every 64-wide K block), 12 TMA for B, 13 TMEM
 // allocation (+ MMA issue in the leader), 14 raw weight stages (codes by TMA,
 // scales by cp.async, 4 K steps per stage) so the dequant warps read only
 // shared memory. Every mbarrier wait is bounded
