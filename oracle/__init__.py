@@ -227,6 +227,99 @@ def quantize_act_int8(x_bf16):
     return q, scale
 
 
+F16_MAX = 65504.0
+
+
+def quantize_h_int8_blocks(h, block: int = 32):
+    """8-bit h for the down projection as a fused SwiGLU quantiser makes it
+    ("Strata NVFP4" README, the 0.1.39-nvfp4.2 bullet: the quantiser keeps its FP16
+    scale finite). Reading taken: blocks of `block` consecutive intermediates, an
+    FP16 scale d = amax / 127 rounded to nearest FP16 and clamped to the largest
+    finite FP16 value, q = nearest integer of h / d (ties to even) clamped to
+    +-127; a zero block has d = 0 and q = 0.
+    h: FP64 [n][I] -> (q int8 [n][I], d f16 [n][I/block])."""
+    h = np.asarray(h, np.float64)
+    n, I = h.shape
+    hb = h.reshape(n, I // block, block)
+    d = np.minimum(np.abs(hb).max(axis=2) / 127.0, F16_MAX).astype(np.float16)
+    d64 = d.astype(np.float64)
+    safe = np.where(d64 > 0, d64, 1.0)
+    q = np.clip(np.rint(hb / safe[:, :, None]), -127, 127)
+    q = np.where(d64[:, :, None] > 0, q, 0).astype(np.int8)
+    return q.reshape(n, I), d
+
+
+def dequant_h_int8_blocks(q, d, block: int = 32) -> np.ndarray:
+    n, I = q.shape
+    return (q.astype(np.float64).reshape(n, I // block, block) *
+            d.astype(np.float64)[:, :, None]).reshape(n, I)
+
+
+def quantize_h_int8_rows(h):
+    """Per-row int8 h: scale = amax / 127 in FP32, q = nearest integer of h / scale
+    (ties to even) clamped to +-127. -> (q int8 [n][I], scale f32 [n])."""
+    h = np.asarray(h, np.float64)
+    s = (np.abs(h).max(axis=1) / 127.0).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float64)
+    return np.clip(np.rint(h / safe[:, None]), -127, 127).astype(np.int8), s
+
+
+_E4M3_POS = None
+
+
+def quantize_h_e4m3_rows(h):
+    """Per-row FP8 h: scale = amax / 448 in FP32 (the row's largest value maps to
+    E4M3's largest finite value), each h / scale rounded to the nearest E4M3 value
+    (ties to the even code), searched over the decoded table of all finite
+    bytes. -> (codes u8 [n][I], scale f32 [n])."""
+    global _E4M3_POS
+    if _E4M3_POS is None:
+        _E4M3_POS = np.array([e4m3(b) for b in range(127)])     # bytes 0x00..0x7E
+    h = np.asarray(h, np.float64)
+    s = (np.abs(h).max(axis=1) / 448.0).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float64)
+    r = np.abs(h) / safe[:, None]
+    dist = np.abs(r[..., None] - _E4M3_POS)
+    best = dist.min(axis=-1, keepdims=True)
+    cand = dist == best
+    # ties: the even byte (a table step is one code apart, so of two equally near
+    # neighbours exactly one is even)
+    even = (np.arange(127) % 2 == 0)
+    pick = np.where(cand.sum(axis=-1) > 1, np.argmax(cand & even, axis=-1), np.argmax(cand, axis=-1))
+    codes = pick.astype(np.uint8) | np.where(h < 0, 0x80, 0).astype(np.uint8)
+    return codes, s
+
+
+def dequant_h_e4m3_rows(codes, s) -> np.ndarray:
+    mag = np.array([e4m3(b) for b in range(128)])[codes & 0x7F]
+    return np.where(codes & 0x80, -mag, mag) * s.astype(np.float64)[:, None]
+
+
+def layer_with_h(layer, x, ids, wts, *, K: int, sample, h_rounds=(None,)) -> list:
+    """Layer outputs, FP64 [n][H] each, for the tokens in `sample`, one per entry of
+    `h_rounds`: each pair's h (the oracle's, FP64) goes through that callable
+    ([n][I] -> [n][I]; None keeps it) before the down projection:
+    out_t = sum_j w_tj * D_e (h_round(h_tj)), D_e decoded with its global. The h
+    of every pair is computed once for all entries; the None entry is `moe`'s
+    result."""
+    xa = _np(x)
+    ia = _np(ids).astype(np.int32)
+    wa = _np(wts).astype(np.float64)
+    dc, ds, dg = (_np(layer.down_codes), _np(layer.down_scales), _np(layer.down_global))
+    D = {}
+    outs = [np.zeros((len(sample), dc.shape[1])) for _ in h_rounds]
+    for n, t in enumerate(sample):
+        hs = np.stack([pair_h(layer, xa[t], int(e), K=K) for e in ia[t]])
+        for out, f in zip(outs, h_rounds):
+            hq = hs if f is None else f(hs)
+            for j, e in enumerate(ia[t]):
+                e = int(e)
+                if e not in D:
+                    D[e] = decode_matrix(dc[e], ds[e], dg[e])
+                out[n] += wa[t, j] * (D[e] @ hq[j])
+    return outs
+
+
 class _Bound:
     """ctypes views of one layer's planes (keeps the numpy arrays alive)."""
 

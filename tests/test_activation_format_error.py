@@ -2,7 +2,9 @@
 block-scaled FP4 x FP4 prompt path (tcgen05 `kind::mxf4nvf4`) or the W4A8 path
 needs them -- the accuracy half of the choice between block-scaled MMA and exact
 dequantisation ("Strata NVFP4" README, "How it differs from upstream Strata", the
-W4A8 bullet: 8-bit activations err far less per product than FP4 ones).
+W4A8 bullet: 8-bit activations err far less per product than FP4 ones) -- and
+when h, between the projections, is stored in 8 bits instead of F16 (the pages'
+fused SwiGLU quantiser, "Strata NVFP4" README, the 0.1.39-nvfp4.2 bullet).
 
 Each variant is evaluated exactly (FP64, dense brute-force formulation of the
 layer) on activations rounded to its format, against the same layer on the BF16
@@ -52,3 +54,28 @@ def test_fp4_activations_miss_the_tolerance_int8_stays_closer(layer, outliers, c
     # 8-bit activations stay closer; with outlier channels a per-token int8 scale
     # spends most of its range on them and keeps less of that advantage
     assert e_i8 < (e_fp4 if outliers else e_fp4 / 5)
+
+
+def test_eight_bit_h_needs_a_looser_tolerance_f16_h_does_not(layer, capsys):
+    T, E, K = 8, 16, 10
+    x = synth.make_x_bf16(T, 2048, seed=31)
+    ids, w = synth.make_topk(T, E, K, seed=33)
+
+    def rows_int8(h):
+        q, s = oracle.quantize_h_int8_rows(h)
+        return q.astype(np.float64) * s.astype(np.float64)[:, None]
+
+    fmts = {
+        "F16": lambda h: h.astype(np.float16).astype(np.float64),
+        "int8, 32-blocks, FP16 scale": lambda h: oracle.dequant_h_int8_blocks(*oracle.quantize_h_int8_blocks(h)),
+        "int8, per row": rows_int8,
+        "E4M3, per row": lambda h: oracle.dequant_h_e4m3_rows(*oracle.quantize_h_e4m3_rows(h)),
+    }
+    outs = oracle.layer_with_h(layer, x, ids, w, K=K, sample=range(T), h_rounds=(None, *fmts.values()))
+    ref = outs[0]
+    err = {name: _rel_l2(o, ref) for name, o in zip(fmts, outs[1:])}
+    with capsys.disabled():
+        print("\n[h formats] layer output rel L2: " + ", ".join(f"{k} {v:.5f}" for k, v in err.items()))
+    assert err["F16"] < TOL_L2 / 5                       # the product's F16 h leaves room
+    assert TOL_L2 < err["int8, 32-blocks, FP16 scale"] < 5 * TOL_L2   # 8-bit h: a 1e-2 bound, not 2e-3
+    assert err["int8, 32-blocks, FP16 scale"] < err["int8, per row"] < err["E4M3, per row"]

@@ -224,6 +224,64 @@ def test_int8_activations_round_trip_and_half_step_bound():
     assert np.all(np.abs(q).max(axis=1) == 127)
 
 
+def test_fp8_h_equals_library_float8_rounding_incl_ties():
+    rng = np.random.default_rng(15)
+    h = rng.standard_normal((4, 96)) * np.array([[1e-3], [1.0], [30.0], [1e4]])
+    c, s = oracle.quantize_h_e4m3_rows(h)
+    r = h / s.astype(np.float64)[:, None]
+    # exact midpoints between neighbouring E4M3 values, both signs: ties go to the even byte
+    pos = np.array([oracle.e4m3(b) for b in range(127)])
+    mids = (pos[1:] + pos[:-1]) / 2.0
+    r2 = np.concatenate([r, np.stack([mids[:96], -mids[20:116]])])
+    r2 = np.clip(r2, -448.0, 448.0)
+    r2[:, 0] = 448.0                                  # keep every row's scale at 1
+    c2, s2 = oracle.quantize_h_e4m3_rows(r2)
+    assert np.all(s2 == 1.0)
+    lib = lambda v: torch.from_numpy(v).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.dequant_h_e4m3_rows(c2, s2), lib(r2))
+    assert np.array_equal(oracle.dequant_h_e4m3_rows(c, s), lib(r) * s.astype(np.float64)[:, None])
+
+
+def test_int8_h_blocks_round_trip_bound_and_finite_fp16_scale():
+    rng = np.random.default_rng(16)
+    q0 = rng.integers(-127, 128, (3, 64))
+    q0[:, 7] = 127
+    q0[:, 40] = -127
+    d0 = np.array([2.0 ** -10, 0.75, 96.0])           # exact in FP16
+    h = (q0.reshape(3, 2, 32) * d0[:, None, None]).reshape(3, 64)
+    q, d = oracle.quantize_h_int8_blocks(h)
+    assert np.array_equal(q.astype(np.int64), q0) and np.array_equal(d.astype(np.float64), np.repeat(d0[:, None], 2, 1))
+    y = rng.standard_normal((5, 96)) * rng.exponential(1.0, (5, 1))
+    q, d = oracle.quantize_h_int8_blocks(y)
+    err = np.abs(oracle.dequant_h_int8_blocks(q, d) - y).reshape(5, 3, 32)
+    dd = d.astype(np.float64)
+    amax = np.abs(y).reshape(5, 3, 32).max(axis=2)
+    assert np.all(np.abs(dd - amax / 127.0) <= np.abs(amax / 127.0) * 2.0 ** -11)   # FP16 nearest
+    # half a step, plus the clamp when rounding d down pushed amax / d past 127
+    assert np.all(err <= (0.5 * dd + np.maximum(amax - 127.0 * dd, 0.0))[:, :, None] * (1 + 1e-12))
+    big = np.full((1, 32), 1e12)
+    big[0, 3] = -1e12
+    q, d = oracle.quantize_h_int8_blocks(big)      # the scale stays finite, the codes saturate
+    assert np.isfinite(d.astype(np.float64)).all() and d[0, 0] == np.float16(65504.0)
+    assert np.all(np.abs(q) == 127) and q[0, 3] == -127
+    q, d = oracle.quantize_h_int8_blocks(np.zeros((1, 32)))
+    assert d[0, 0] == 0 and not q.any()
+    q, s = oracle.quantize_h_int8_rows(h)
+    assert np.all(np.abs(q).max(axis=1) == 127)
+    assert np.all(np.abs(q * s.astype(np.float64)[:, None] - h) <= 0.5 * s.astype(np.float64)[:, None] * (1 + 1e-6))
+
+
+def test_layer_with_h_unrounded_is_the_oracle_layer():
+    d = synth.LayerDims(E=6, H=64, I=48, K=3)
+    layer = synth.make_layer(d, seed=17)
+    x = synth.make_x_bf16(5, 64, seed=18)
+    ids, w = synth.make_topk(5, 6, 3, seed=19)
+    ref = oracle.moe(layer, x, ids, w.double(), K=3)
+    out, neg = oracle.layer_with_h(layer, x, ids, w, K=3, sample=range(5), h_rounds=(None, lambda h: -h))
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    np.testing.assert_allclose(neg, -ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())   # linear in h
+
+
 # ----------------------------------------------------------------- routing
 
 def test_route_matches_library_sort_and_softmax():
