@@ -45,8 +45,7 @@
  *     valid until nvfp4_moe_destroy. The library allocates no device memory
  *     except what nvfp4_moe_create makes: a 256-byte status block and, when
  *     the layer can take the decode kernel, its state, kept zero between calls:
- *     a counter and a 64-bit copy of the output, 256 + 64 * H bytes (128 KB for
- *     H = 2048).
+ *     the counters of its grid barrier, 256 bytes.
  *   - All other scratch lives in the caller's workspace (nvfp4_moe_workspace_bytes).
  *
  * Errors: every call returns 0 (NVFP4_MOE_OK) or a negative nvfp4_moe_status.
@@ -279,7 +278,7 @@ NVFP4_MOE_API int nvfp4_moe_set_phase_events(nvfp4_moe_t *h, void *const *events
  *     returns NVFP4_MOE_ERR_UNSUPPORTED_DIMS; a layer whose decode scratch and
  *     state for this T exceed 1 MiB - 256 bytes would return
  *     NVFP4_MOE_ERR_WORKSPACE_TOO_SMALL (no layer the decode kernel takes needs
- *     that much: its state is 64 * H bytes and its shared memory bounds H and
+ *     that much: its state is 256 bytes and its shared memory bounds H and
  *     the expert count). Both are checked before anything is enqueued. T = 0
  *     is a no-op.
  *   - The first call on a device does a one-time set-up there: it looks up the
