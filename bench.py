@@ -268,8 +268,9 @@ def run_ours(args, ws, rank, local):
     flops_dn = 2.0 * P * d.H * d.I
     gu_ms = phase_ms[2]
     achieved = flops_gu / (gu_ms / 1e3) / 1e12
-    # The sampled SM clock stays within a few percent of its maximum during the
-    # step (sw_power_cap is flagged but barely lowers it), so the burst cuBLAS figure
+    # The sampled SM clock stays within about 10 % of its maximum during the
+    # step (sw_power_cap is flagged; far above the ~1.3 GHz of a seconds-long
+    # GEMM loop), so the burst cuBLAS figure
     # is the denominator; the sustained one is context.
     peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     # The gate/up phase is two launches: the tensor-core tiles of the experts with
