@@ -328,6 +328,8 @@ def test_sort_matches_stable_library_sort():
     assert counts.sum() == 300 * 6 and np.array_equal(np.bincount(flat, minlength=40), counts)
     assert np.array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
     assert np.array_equal(np.sort(perm), np.arange(300 * 6))
+    assert np.all(np.bincount(perm // 6, minlength=300) == 6)   # every token K times
+    assert np.all(np.diff(flat[perm]) >= 0)                     # grouped by expert ascending
 
 
 def test_check_ids():
