@@ -79,3 +79,21 @@ def test_eight_bit_h_needs_a_looser_tolerance_f16_h_does_not(layer, capsys):
     assert err["F16"] < TOL_L2 / 5                       # the product's F16 h leaves room
     assert TOL_L2 < err["int8, 32-blocks, FP16 scale"] < 5 * TOL_L2   # 8-bit h: a 1e-2 bound, not 2e-3
     assert err["int8, 32-blocks, FP16 scale"] < err["int8, per row"] < err["E4M3, per row"]
+
+
+@pytest.mark.parametrize("outliers", [False, True])
+def test_eight_bit_blocks_err_about_sixteen_times_less_than_fp4(outliers, capsys):
+    # The pages put the W4A8 path's 8-bit activations at 16x smaller error per
+    # product than FP4 ones ("Strata NVFP4" README, "How it differs from upstream
+    # Strata", the W4A8 bullet). The 8-bit format read as llama.cpp's: blocks of
+    # 32 with an FP16 scale; FP4 as per-token NVFP4. A product's error from its
+    # activation is that activation's rounding error, so the ratio of the two
+    # formats' element errors is the figure to compare.
+    x = synth.make_x_bf16(24, 2048, seed=22 + outliers, outliers=outliers)
+    x64 = brute.bf16_to_f64(x)
+    x8 = oracle.dequant_h_int8_blocks(*oracle.quantize_h_int8_blocks(x64))
+    x4 = oracle.dequant_act_nvfp4(*oracle.quantize_act_nvfp4(x))
+    ratio = _rel_l2(x4, x64) / _rel_l2(x8, x64)
+    with capsys.disabled():
+        print(f"\n[8-bit vs FP4 activations, outliers={outliers}] element error ratio {ratio:.1f}")
+    assert 8.0 < ratio < 32.0
