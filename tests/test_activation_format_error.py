@@ -97,3 +97,29 @@ def test_eight_bit_blocks_err_about_sixteen_times_less_than_fp4(outliers, capsys
     with capsys.disabled():
         print(f"\n[8-bit vs FP4 activations, outliers={outliers}] element error ratio {ratio:.1f}")
     assert 8.0 < ratio < 32.0
+
+
+def test_single_expert_with_eight_bit_blocks_brackets_the_pages_parity_error(capsys):
+    # The pages report a three-expert CUDA parity of 1.096 %, 1.156 % and 1.159 %
+    # relative output error against a 3 % threshold ("#2727 tools: add opt-in
+    # FP4-Local CSF checkpoint conversion", "Validation") without saying what the
+    # reference is. One plausible reading: their prompt path's 8-bit activations
+    # (32-blocks, FP16 scales) against a float reference. One expert of the
+    # benchmark shape, exact otherwise, with and without outlier channels:
+    layer = synth.make_layer(synth.LayerDims(E=3, H=2048, I=768, K=1), seed=41)
+    errs = {}
+    for outliers in (False, True):
+        x = synth.make_x_bf16(32, 2048, seed=42 + outliers, outliers=outliers)
+        x64 = brute.bf16_to_f64(x)
+        x8 = oracle.dequant_h_int8_blocks(*oracle.quantize_h_int8_blocks(x64))
+        for e in range(3):
+            G = np.zeros((32, 3))
+            G[:, e] = 1.0
+            o = brute.layer_out(layer, np.concatenate([x64, x8]), np.concatenate([G, G]))
+            errs[(outliers, e)] = _rel_l2(o[32:], o[:32])
+    with capsys.disabled():
+        print("\n[one expert, 8-bit block activations] rel L2: " +
+              ", ".join(f"{'outliers' if k[0] else 'plain'} e{k[1]} {100 * v:.2f} %" for k, v in errs.items()))
+    plain = [v for k, v in errs.items() if not k[0]]
+    outl = [v for k, v in errs.items() if k[0]]
+    assert max(plain) < 0.011 < min(outl) and max(outl) < 0.03   # brackets 1.1 %, under the 3 % threshold
