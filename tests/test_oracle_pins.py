@@ -247,10 +247,10 @@ def test_int8_h_blocks_round_trip_bound_and_finite_fp16_scale():
     q0 = rng.integers(-127, 128, (3, 64))
     q0[:, 7] = 127
     q0[:, 40] = -127
-    d0 = np.array([2.0 ** -10, 0.75, 96.0])           # exact in FP16
-    h = (q0.reshape(3, 2, 32) * d0[:, None, None]).reshape(3, 64)
+    d0 = np.array([[2.0 ** -10, 3.0], [0.75, 2.0 ** -3], [96.0, 0.5]])   # exact in FP16, one per block
+    h = (q0.reshape(3, 2, 32) * d0[:, :, None]).reshape(3, 64)
     q, d = oracle.quantize_h_int8_blocks(h)
-    assert np.array_equal(q.astype(np.int64), q0) and np.array_equal(d.astype(np.float64), np.repeat(d0[:, None], 2, 1))
+    assert np.array_equal(q.astype(np.int64), q0) and np.array_equal(d.astype(np.float64), d0)
     y = rng.standard_normal((5, 96)) * rng.exponential(1.0, (5, 1))
     q, d = oracle.quantize_h_int8_blocks(y)
     err = np.abs(oracle.dequant_h_int8_blocks(q, d) - y).reshape(5, 3, 32)
